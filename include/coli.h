@@ -1,0 +1,164 @@
+/*
+ * coli.h -- C ABI of the B200 routed-expert MoE layer library (libcoli.so).
+ *
+ * The calls follow the colibri pages' per-token path: Route, then Union, then
+ * the expert compute with its combine (Korean getting-started page, section
+ * 토큰당 처리 경로 "The Per-Token Path"; "colibri: 744B MoEをストレージから推論する
+ * Cエンジン", section トークンごとの5ステップパスとデュアルSSDミラー).  The two
+ * steps of that path about storage (Place, Learn) have no counterpart here:
+ * every expert is resident in HBM.
+ *
+ * Conventions for every call:
+ *   - Every tensor pointer is a caller-owned DEVICE pointer, row-major and
+ *     densely packed.  The library allocates no device memory and keeps no
+ *     device state between calls; scratch memory is the caller's workspace.
+ *   - All work is enqueued on the given stream; calls are asynchronous and
+ *     never synchronise the device.  Argument checks run on the host before
+ *     anything is enqueued: a call that returns an error has launched nothing.
+ *   - Nothing is thrown across the ABI.  Every call returns a coli_status;
+ *     coli_last_error() returns a description of the calling thread's most
+ *     recent failure.
+ *   - Sizes: hidden H and expert width F are multiples of 64 (the int4 group),
+ *     H and F <= 16384; 1 <= top_k <= 32; top_k <= n_experts <= 1024;
+ *     0 <= T <= 65536.  T == 0 is a valid empty call: coli_router_topk and
+ *     coli_moe_forward launch nothing, coli_expert_union still writes its
+ *     per-expert outputs (all counts zero).
+ *   - Alignment: activations, outputs and weight/scale pointers 16-byte
+ *     aligned; workspace 256-byte aligned.
+ *
+ * int4-gs64 storage of one matrix [N, K] ("gs64 build" of the int4 container,
+ * "colibri: 744B MoE…", section はじめにとソースが語らないこと): bytes [N, K/2],
+ * two values per byte, even k in the low nibble, each nibble a two's-complement
+ * integer in [-8, 7] with no zero point; fp32 scales [N, K/64];
+ * W[n, k] = q[n, k] * scale[n, k / 64].
+ */
+#ifndef COLI_H
+#define COLI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define COLI_API __attribute__((visibility("default")))
+#else
+#define COLI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    COLI_OK = 0,
+    COLI_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or dtype */
+    COLI_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    COLI_ERR_WORKSPACE = 3,    /* workspace smaller than coli_moe_workspace_size() */
+    COLI_ERR_CUDA = 4          /* a CUDA runtime call failed; see coli_last_error() */
+} coli_status;
+
+typedef enum { COLI_F32 = 0, COLI_BF16 = 1 } coli_dtype;
+
+/* One MoE layer.  Expert index n_experts is the shared expert, so every
+ * expert array holds n_experts + 1 experts, expert-major. */
+typedef struct {
+    int hidden;            /* H, e.g. 6144 */
+    int ffn;               /* F, expert width, e.g. 2048 */
+    int n_experts;         /* E routed experts, e.g. 256 */
+    int top_k;             /* k, e.g. 8 */
+    int group;             /* scale group along K; must be 64 */
+    float routed_scale;    /* factor applied to the renormalised routed weights, e.g. 2.5 */
+    const float* w_router; /* [E, H] fp32 */
+    const float* sel_bias; /* [E] fp32, selection-only bias */
+    const uint8_t* gate_q; /* [E+1, F, H/2] */
+    const uint8_t* up_q;   /* [E+1, F, H/2] */
+    const uint8_t* down_q; /* [E+1, H, F/2] */
+    const float* gate_s;   /* [E+1, F, H/64] */
+    const float* up_s;     /* [E+1, F, H/64] */
+    const float* down_s;   /* [E+1, H, F/64] */
+} coli_moe_layer;
+
+/*
+ * Route ("Colibri 完全ガイド", section コア技術のハイライト: DeepSeek-V3-style
+ * sigmoid router).  For each token t of x [T, H] (dtype xt):
+ *   logit_e = x_t . w_router[e];  s_e = 1/(1+exp(-logit_e));  c_e = s_e + sel_bias[e]
+ *   topk_idx[t, :] = the k experts of largest c_e, in descending c_e
+ *                    (equal c_e: lower expert index first)
+ *   topk_w[t, j]   = routed_scale * s_idx[j] / sum_j' s_idx[j']
+ * The bias selects experts but does not enter the weights.  Computed in fp32.
+ * Outputs: topk_idx int32 [T, k], topk_w fp32 [T, k] (device).
+ */
+COLI_API coli_status coli_router_topk(const void* x, coli_dtype xt, int T, int H,
+                             const float* w_router, const float* sel_bias, int E, int k,
+                             float routed_scale, int32_t* topk_idx, float* topk_w,
+                             cudaStream_t stream);
+
+/*
+ * Union (Korean getting-started page, section 토큰당 처리 경로, "Union": experts
+ * chosen by several tokens of the batch are de-duplicated).  A stable counting
+ * sort of the T*k pairs p = t*k + j by expert topk_idx[p]:
+ *   count[E]      pairs per expert
+ *   offset[E+1]   exclusive prefix sum of count (offset[E] = T*k)
+ *   active[E]     experts with count > 0 in ascending order, tail filled with -1
+ *   n_active[1]   number of active experts (the batch union size U)
+ *   perm[T*k]     pair ids in (expert, token, slot) order
+ *   inv_perm[T*k] inv_perm[perm[i]] = i
+ * All outputs are int32 device arrays; results are deterministic (bit-exact).
+ * Every topk_idx entry must lie in [0, E); this is not checked on the device.
+ */
+COLI_API coli_status coli_expert_union(const int32_t* topk_idx, int T, int k, int E,
+                              int32_t* count, int32_t* offset, int32_t* active,
+                              int32_t* n_active, int32_t* perm, int32_t* inv_perm,
+                              cudaStream_t stream);
+
+/* Bytes of workspace coli_moe_forward needs for T tokens of this layer
+ * (0 if the layer description is invalid). */
+COLI_API size_t coli_moe_workspace_size(const coli_moe_layer* layer, int T);
+
+/*
+ * The whole layer: Route, Union, the expert FFNs and the weighted combine.
+ *   out_t = sum_j topk_w[t,j] * FFN_{topk_idx[t,j]}(x_t) + FFN_shared(x_t)
+ *   FFN_e(x) = W_down,e (silu(W_gate,e x) * (W_up,e x)),  silu(z) = z/(1+exp(-z))
+ * The pages name the routed experts, the shared expert ("Colibri 完全ガイド",
+ * DeepSeek-V3 router row) and int4 weights with one scale per 64; the SwiGLU
+ * form of the expert and the unscaled, always-on shared expert are this
+ * library's reading of them.  Activations and accumulation are fp32 (bf16 x is
+ * widened exactly); out is written as fp32 or bf16 (round to nearest even).
+ * x [T, H] dtype xt; out [T, H] dtype ot; workspace of at least
+ * coli_moe_workspace_size(layer, T) bytes, contents undefined on entry and
+ * exit, not shared by calls that may run concurrently.  topk_idx_out [T, k]
+ * and topk_w_out [T, k] are optional copies of the routing (NULL to skip).
+ */
+COLI_API coli_status coli_moe_forward(const coli_moe_layer* layer, const void* x, coli_dtype xt, int T,
+                             void* out, coli_dtype ot, void* workspace, size_t ws_bytes,
+                             int32_t* topk_idx_out, float* topk_w_out, cudaStream_t stream);
+
+/* Stages of coli_moe_forward, for coli_moe_profile_next(). */
+enum {
+    COLI_STAGE_ROUTE = 0,   /* router scores and top-k */
+    COLI_STAGE_UNION = 1,   /* batch union and work lists */
+    COLI_STAGE_GATEUP = 2,  /* gate/up projections with SwiGLU */
+    COLI_STAGE_DOWN = 3,    /* down projections, routing weight applied */
+    COLI_STAGE_COMBINE = 4, /* per-token sum of expert outputs into out */
+    COLI_N_STAGES = 5
+};
+
+/*
+ * Optional stage timing.  Arms a one-shot hook for the calling host thread:
+ * the next coli_moe_forward on this thread records events[2*s] on its stream
+ * just before stage s and events[2*s+1] just after it, for s < n_events/2,
+ * then disarms.  Stages that a path fuses into another are recorded
+ * back-to-back.  events are caller-created cudaEvent_t handles (host objects);
+ * pass events = NULL to disarm.  Inside stream capture the records become
+ * external event-record nodes of the graph.
+ */
+COLI_API coli_status coli_moe_profile_next(cudaEvent_t* events, int n_events);
+
+COLI_API const char* coli_status_string(coli_status status);
+COLI_API const char* coli_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COLI_H */

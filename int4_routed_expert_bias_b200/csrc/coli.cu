@@ -1,0 +1,381 @@
+// coli.cu -- C ABI of the routed-expert MoE layer (see include/coli.h).
+//
+// Host side: argument checks (before anything is enqueued), workspace layout,
+// kernel selection and launch order.  Every step of the layer runs in the
+// kernels of this library; there is no CPU fallback.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "coli.h"
+#include "coli_common.cuh"
+#include "coli_decode.cuh"
+#include "coli_router.cuh"
+#include "coli_union.cuh"
+
+using namespace coli;
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local cudaEvent_t* g_prof_events = nullptr;
+thread_local int g_prof_n = 0;
+
+coli_status fail(coli_status st, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+coli_status cuda_fail(cudaError_t e, const char* what)
+{
+    return fail(COLI_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+constexpr int kMaxTokens = 65536;
+
+coli_status check_sizes(int T, int H, int E, int k)
+{
+    if (T < 0 || T > kMaxTokens) return fail(COLI_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, kMaxTokens);
+    if (H <= 0 || H % kGroup != 0) return fail(COLI_ERR_INVALID_ARG, "hidden=%d is not a positive multiple of 64", H);
+    if (k < 1 || k > kMaxTopK) return fail(COLI_ERR_INVALID_ARG, "top_k=%d outside [1, %d]", k, kMaxTopK);
+    if (E < k || E > kMaxExperts) return fail(COLI_ERR_INVALID_ARG, "n_experts=%d outside [top_k=%d, %d]", E, k, kMaxExperts);
+    return COLI_OK;
+}
+
+// Per-device launch facts, filled on first use: SM count, and the dynamic
+// shared-memory limit that every staged-activation kernel is opted in to.
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int smem_optin = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+constexpr int kMaxStageK = 16384;  // largest hidden / ffn width accepted
+size_t gateup_smem(int H, int TG) { return stage_smem_bytes(H, TG); }
+size_t down_smem(int F, int TG) { return stage_smem_bytes(F, TG); }
+
+template <typename Kern>
+cudaError_t allow_smem(Kern k, int bytes)
+{
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+coli_status device_info(DeviceInfo** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(COLI_ERR_UNSUPPORTED, "device %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        const int lim = d.smem_optin - 1024;  // room for the kernels' static shared memory
+        if ((e = allow_smem(expert_phase_kernel<true, false, 1>, lim)) != cudaSuccess ||
+            (e = allow_smem(expert_phase_kernel<true, false, 4>, lim)) != cudaSuccess ||
+            (e = allow_smem(expert_phase_kernel<true, true, 1>, lim)) != cudaSuccess ||
+            (e = allow_smem(expert_phase_kernel<true, true, 4>, lim)) != cudaSuccess ||
+            (e = allow_smem(expert_phase_kernel<false, false, 1>, lim)) != cudaSuccess ||
+            (e = allow_smem(expert_phase_kernel<false, false, 4>, lim)) != cudaSuccess)
+            return cuda_fail(e, "kernel attribute setup");
+        d.smem_optin = lim;
+        d.ready = true;
+    }
+    *out = &d;
+    return COLI_OK;
+}
+
+// Resident blocks per SM for the actual dynamic smem of one launch.
+template <typename Kern>
+int blocks_per_sm(Kern k, size_t smem)
+{
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kDecThreads, smem) != cudaSuccess) return 1;
+    return occ > 0 ? occ : 1;
+}
+
+// Tokens per group of the expert phases: 4 when the staged activations fit.
+int group_tokens(int T, int H, int F, int smem_limit)
+{
+    if (T == 1) return 1;
+    if (gateup_smem(H, 4) <= (size_t)smem_limit && down_smem(F, 4) <= (size_t)smem_limit) return 4;
+    return 1;
+}
+
+// ---------------------------------------------------------------------------
+// workspace layout
+
+struct Workspace {
+    float* logits;      // [T, E]
+    int32_t* idx;       // [P]
+    float* w;           // [P]
+    int32_t* count;     // [E]
+    int32_t* offset;    // [E+1]
+    int32_t* active;    // [E]
+    int32_t* n_active;  // [1]
+    int32_t* perm;      // [P]
+    int32_t* inv_perm;  // [P]
+    int32_t* pair_token;  // [P+T]
+    float* pair_w;        // [P+T]
+    int32_t* ctl;         // [4]
+    int32_t* g_expert;    // [G]
+    int32_t* g_start;
+    int32_t* g_count;
+    float* h;             // [P+T, F]
+    float* partial;       // [P+T, H]
+    size_t bytes;
+};
+
+Workspace layout(void* base, int T, int H, int F, int E, int k)
+{
+    Workspace w{};
+    const size_t P = (size_t)T * k, Q = P + T, G = P + (size_t)E + T + 1;
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char* {
+        char* p = base ? static_cast<char*>(base) + off : nullptr;
+        off += align_up(bytes, 256);
+        return p;
+    };
+    w.logits = (float*)take((size_t)T * E * 4);
+    w.idx = (int32_t*)take(P * 4);
+    w.w = (float*)take(P * 4);
+    w.count = (int32_t*)take((size_t)E * 4);
+    w.offset = (int32_t*)take(((size_t)E + 1) * 4);
+    w.active = (int32_t*)take((size_t)E * 4);
+    w.n_active = (int32_t*)take(4);
+    w.perm = (int32_t*)take(P * 4);
+    w.inv_perm = (int32_t*)take(P * 4);
+    w.pair_token = (int32_t*)take(Q * 4);
+    w.pair_w = (float*)take(Q * 4);
+    w.ctl = (int32_t*)take(16);
+    w.g_expert = (int32_t*)take(G * 4);
+    w.g_start = (int32_t*)take(G * 4);
+    w.g_count = (int32_t*)take(G * 4);
+    w.h = (float*)take(Q * F * 4);
+    w.partial = (float*)take(Q * H * 4);
+    w.bytes = off;
+    return w;
+}
+
+coli_status check_layer(const coli_moe_layer* L, int T)
+{
+    if (!L) return fail(COLI_ERR_INVALID_ARG, "layer is NULL");
+    coli_status st = check_sizes(T, L->hidden, L->n_experts, L->top_k);
+    if (st != COLI_OK) return st;
+    if (L->ffn <= 0 || L->ffn % kGroup != 0) return fail(COLI_ERR_INVALID_ARG, "ffn=%d is not a positive multiple of 64", L->ffn);
+    if (L->group != kGroup) return fail(COLI_ERR_UNSUPPORTED, "group=%d (only 64 is supported)", L->group);
+    if (L->hidden > kMaxStageK || L->ffn > kMaxStageK)
+        return fail(COLI_ERR_UNSUPPORTED, "hidden=%d / ffn=%d above %d", L->hidden, L->ffn, kMaxStageK);
+    if (!std::isfinite(L->routed_scale)) return fail(COLI_ERR_INVALID_ARG, "routed_scale is not finite");
+    const void* ptrs[] = {L->w_router, L->sel_bias, L->gate_q, L->up_q, L->down_q, L->gate_s, L->up_s, L->down_s};
+    const char* names[] = {"w_router", "sel_bias", "gate_q", "up_q", "down_q", "gate_s", "up_s", "down_s"};
+    for (int i = 0; i < 8; ++i) {
+        if (!ptrs[i]) return fail(COLI_ERR_INVALID_ARG, "layer.%s is NULL", names[i]);
+        if (!aligned(ptrs[i], i == 1 ? 4 : 16)) return fail(COLI_ERR_INVALID_ARG, "layer.%s is not 16-byte aligned", names[i]);
+    }
+    return COLI_OK;
+}
+
+struct StageTimer {
+    cudaEvent_t* ev = nullptr;
+    int n = 0;
+    bool capturing = false;
+    cudaStream_t s = nullptr;
+    cudaError_t rec(int stage, int end)
+    {
+        const int i = 2 * stage + end;
+        if (!ev || i >= n) return cudaSuccess;
+        return capturing ? cudaEventRecordWithFlags(ev[i], s, cudaEventRecordExternal) : cudaEventRecord(ev[i], s);
+    }
+};
+
+coli_status launch_route(const void* x, coli_dtype xt, int T, int H, const float* w_router,
+                         const float* sel_bias, int E, int k, float routed_scale, float* logits,
+                         int32_t* idx, float* w, cudaStream_t s)
+{
+    dim3 grid(E, (T + kRouterTokens - 1) / kRouterTokens);
+    if (xt == COLI_BF16) router_logits_kernel<true><<<grid, kRouterThreads, 0, s>>>(x, T, H, w_router, E, logits);
+    else router_logits_kernel<false><<<grid, kRouterThreads, 0, s>>>(x, T, H, w_router, E, logits);
+    const int warps_per_block = 8;
+    router_topk_kernel<<<(T + warps_per_block - 1) / warps_per_block, 256, 0, s>>>(
+        logits, T, E, k, sel_bias, routed_scale, idx, w);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? COLI_OK : cuda_fail(e, "router launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* coli_status_string(coli_status st)
+{
+    switch (st) {
+        case COLI_OK: return "COLI_OK";
+        case COLI_ERR_INVALID_ARG: return "COLI_ERR_INVALID_ARG";
+        case COLI_ERR_UNSUPPORTED: return "COLI_ERR_UNSUPPORTED";
+        case COLI_ERR_WORKSPACE: return "COLI_ERR_WORKSPACE";
+        case COLI_ERR_CUDA: return "COLI_ERR_CUDA";
+    }
+    return "COLI_ERR_UNKNOWN";
+}
+
+const char* coli_last_error(void) { return g_err; }
+
+coli_status coli_moe_profile_next(cudaEvent_t* events, int n_events)
+{
+    if (events && n_events < 0) return fail(COLI_ERR_INVALID_ARG, "n_events < 0");
+    g_prof_events = events;
+    g_prof_n = events ? n_events : 0;
+    return COLI_OK;
+}
+
+coli_status coli_router_topk(const void* x, coli_dtype xt, int T, int H, const float* w_router,
+                             const float* sel_bias, int E, int k, float routed_scale,
+                             int32_t* topk_idx, float* topk_w, cudaStream_t stream)
+{
+    coli_status st = check_sizes(T, H, E, k);
+    if (st != COLI_OK) return st;
+    if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown activation dtype %d", (int)xt);
+    if (T == 0) return COLI_OK;
+    if (!x || !w_router || !sel_bias || !topk_idx || !topk_w) return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(x, 16) || !aligned(w_router, 16)) return fail(COLI_ERR_INVALID_ARG, "x / w_router not 16-byte aligned");
+    if (!std::isfinite(routed_scale)) return fail(COLI_ERR_INVALID_ARG, "routed_scale is not finite");
+    dim3 grid(kRouterCluster * ((T + kRouterTokens - 1) / kRouterTokens));
+    if (xt == COLI_BF16)
+        router_cluster_kernel<true><<<grid, kRouterClusterThreads, 0, stream>>>(
+            x, T, H, w_router, sel_bias, E, k, routed_scale, topk_idx, topk_w);
+    else
+        router_cluster_kernel<false><<<grid, kRouterClusterThreads, 0, stream>>>(
+            x, T, H, w_router, sel_bias, E, k, routed_scale, topk_idx, topk_w);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? COLI_OK : cuda_fail(e, "router launch");
+}
+
+coli_status coli_expert_union(const int32_t* topk_idx, int T, int k, int E, int32_t* count,
+                              int32_t* offset, int32_t* active, int32_t* n_active, int32_t* perm,
+                              int32_t* inv_perm, cudaStream_t stream)
+{
+    if (T < 0 || T > kMaxTokens) return fail(COLI_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, kMaxTokens);
+    if (k < 1 || k > kMaxTopK) return fail(COLI_ERR_INVALID_ARG, "top_k=%d outside [1, %d]", k, kMaxTopK);
+    if (E < k || E > kMaxExperts) return fail(COLI_ERR_INVALID_ARG, "n_experts=%d outside [top_k, %d]", E, kMaxExperts);
+    if (!count || !offset || !active || !n_active || (T > 0 && (!topk_idx || !perm || !inv_perm)))
+        return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
+    WorkLists wl{};
+    union_kernel<false><<<1, kUnionThreads, 0, stream>>>(topk_idx, T, k, E, count, offset, active,
+                                                         n_active, perm, inv_perm, wl);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? COLI_OK : cuda_fail(e, "union launch");
+}
+
+size_t coli_moe_workspace_size(const coli_moe_layer* L, int T)
+{
+    if (check_layer(L, T) != COLI_OK) return 0;
+    return layout(nullptr, T, L->hidden, L->ffn, L->n_experts, L->top_k).bytes;
+}
+
+coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype xt, int T, void* out,
+                             coli_dtype ot, void* workspace, size_t ws_bytes, int32_t* topk_idx_out,
+                             float* topk_w_out, cudaStream_t stream)
+{
+    StageTimer tm;
+    tm.ev = g_prof_events;
+    tm.n = g_prof_n;
+    g_prof_events = nullptr;  // one-shot
+    g_prof_n = 0;
+
+    coli_status st = check_layer(L, T);
+    if (st != COLI_OK) return st;
+    if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown activation dtype %d", (int)xt);
+    if (ot != COLI_F32 && ot != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown output dtype %d", (int)ot);
+    if (T == 0) return COLI_OK;
+    if (!x || !out || !workspace) return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(x, 16) || !aligned(out, 16)) return fail(COLI_ERR_INVALID_ARG, "x / out not 16-byte aligned");
+    if (!aligned(workspace, 256)) return fail(COLI_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    if ((topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
+        return fail(COLI_ERR_INVALID_ARG, "routing outputs not 4-byte aligned");
+    const int H = L->hidden, F = L->ffn, E = L->n_experts, k = L->top_k;
+    Workspace w = layout(workspace, T, H, F, E, k);
+    if (ws_bytes < w.bytes)
+        return fail(COLI_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, w.bytes);
+
+    DeviceInfo* dev = nullptr;
+    if ((st = device_info(&dev)) != COLI_OK) return st;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    tm.capturing = (cs == cudaStreamCaptureStatusActive);
+    tm.s = stream;
+
+    int32_t* idx = topk_idx_out ? topk_idx_out : w.idx;
+    float* wt = topk_w_out ? topk_w_out : w.w;
+    const int TG = group_tokens(T, H, F, dev->smem_optin);
+    const bool bf16 = (xt == COLI_BF16);
+
+    // Route
+    if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
+    st = launch_route(x, xt, T, H, L->w_router, L->sel_bias, E, k, L->routed_scale, w.logits, idx, wt, stream);
+    if (st != COLI_OK) return st;
+    if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    // Union and work lists
+    if ((e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess) return cuda_fail(e, "event record");
+    WorkLists wl{w.pair_token, w.pair_w, w.ctl, w.g_expert, w.g_start, w.g_count, wt, TG};
+    union_kernel<true><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
+                                                        w.n_active, w.perm, w.inv_perm, wl);
+    if ((e = tm.rec(COLI_STAGE_UNION, 1)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    // Gate/up + SwiGLU for every token group (routed experts, then the shared expert)
+    PhaseArgs ga{L->gate_q, L->gate_s, L->up_q, L->up_s, F, H, x, w.ctl, w.ctl + 1,
+                 w.g_expert, w.g_start, w.g_count, w.pair_token, w.pair_w, w.h};
+    const size_t gsm = gateup_smem(H, TG);
+    if ((e = tm.rec(COLI_STAGE_GATEUP, 0)) != cudaSuccess) return cuda_fail(e, "event record");
+    {
+        auto kern = bf16 ? (TG == 1 ? expert_phase_kernel<true, true, 1> : expert_phase_kernel<true, true, 4>)
+                         : (TG == 1 ? expert_phase_kernel<true, false, 1> : expert_phase_kernel<true, false, 4>);
+        const int grid = dev->sms * blocks_per_sm(kern, gsm);
+        kern<<<grid, kDecThreads, gsm, stream>>>(ga);
+    }
+    if ((e = tm.rec(COLI_STAGE_GATEUP, 1)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    // Down projection with the routing weight, one partial row per pair
+    PhaseArgs da{L->down_q, L->down_s, nullptr, nullptr, H, F, w.h, w.ctl, w.ctl + 2,
+                 w.g_expert, w.g_start, w.g_count, w.pair_token, w.pair_w, w.partial};
+    const size_t dsm = down_smem(F, TG);
+    if ((e = tm.rec(COLI_STAGE_DOWN, 0)) != cudaSuccess) return cuda_fail(e, "event record");
+    {
+        auto kern = TG == 1 ? expert_phase_kernel<false, false, 1> : expert_phase_kernel<false, false, 4>;
+        const int grid = dev->sms * blocks_per_sm(kern, dsm);
+        kern<<<grid, kDecThreads, dsm, stream>>>(da);
+    }
+    if ((e = tm.rec(COLI_STAGE_DOWN, 1)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    // Combine
+    if ((e = tm.rec(COLI_STAGE_COMBINE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
+    {
+        const int n = T * (H / 4);
+        const int blocks = (n + 255) / 256;
+        if (ot == COLI_BF16) combine_kernel<true><<<blocks, 256, 0, stream>>>(w.partial, w.inv_perm, T, k, H, out);
+        else combine_kernel<false><<<blocks, 256, 0, stream>>>(w.partial, w.inv_perm, T, k, H, out);
+    }
+    if ((e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    e = cudaGetLastError();
+    return e == cudaSuccess ? COLI_OK : cuda_fail(e, "layer launch");
+}
+
+}  // extern "C"

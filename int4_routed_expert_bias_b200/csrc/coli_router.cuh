@@ -1,0 +1,198 @@
+// coli_router.cuh -- Route: router scores (fp32 GEMV) and bias-corrected top-k.
+//
+// DeepSeek-V3-style sigmoid router ("Colibri 完全ガイド", section コア技術のハイライト):
+//   logit_e = x . w_router[e], s_e = sigmoid(logit_e), c_e = s_e + bias_e,
+//   idx = top-k of c (descending, equal c -> lower e), w_j = alpha * s_j / sum s.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "coli_common.cuh"
+
+namespace coli {
+
+constexpr int kRouterTokens = 4;     // tokens per router block
+constexpr int kRouterThreads = 256;
+
+// logits[t, e] for one expert row e (blockIdx.x) and up to kRouterTokens tokens
+// (blockIdx.y).  The row of w_router is read once per token group with 16-byte
+// loads; the per-thread partial sums are reduced in a fixed order, so the
+// result is deterministic.
+template <bool kBf16>
+__global__ void __launch_bounds__(kRouterThreads)
+router_logits_kernel(const void* __restrict__ x, int T, int H, const float* __restrict__ w_router,
+                     int E, float* __restrict__ logits)
+{
+    const int e = blockIdx.x;
+    const int t0 = blockIdx.y * kRouterTokens;
+    const int nt = min(kRouterTokens, T - t0);
+    const float* wrow = w_router + (size_t)e * H;
+    const size_t xrow_bytes = (size_t)H * (kBf16 ? 2 : 4);
+    const char* xb = static_cast<const char*>(x) + (size_t)t0 * xrow_bytes;
+
+    float acc[kRouterTokens];
+#pragma unroll
+    for (int t = 0; t < kRouterTokens; ++t) acc[t] = 0.f;
+
+    for (int i = threadIdx.x * 4; i < H; i += kRouterThreads * 4) {
+        const float4 w = *reinterpret_cast<const float4*>(wrow + i);
+#pragma unroll
+        for (int t = 0; t < kRouterTokens; ++t) {
+            if (t < nt) {
+                const float4 v = load_act4<kBf16>(xb + t * xrow_bytes, i);
+                acc[t] = fmaf(w.x, v.x, acc[t]);
+                acc[t] = fmaf(w.y, v.y, acc[t]);
+                acc[t] = fmaf(w.z, v.z, acc[t]);
+                acc[t] = fmaf(w.w, v.w, acc[t]);
+            }
+        }
+    }
+    __shared__ float red[kRouterThreads / 32][kRouterTokens];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int t = 0; t < kRouterTokens; ++t) {
+        const float v = warp_sum(acc[t]);
+        if (lane == 0) red[warp][t] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < nt) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kRouterThreads / 32; ++w) v += red[w][threadIdx.x];
+        logits[(size_t)(t0 + threadIdx.x) * E + e] = v;
+    }
+}
+
+// Top-k of one token by one warp: sigmoid, bias, k rounds of warp arg-max,
+// renormalised weights.  Lane j keeps the j-th selection.  The arg-max key is
+// (c desc, index asc); a non-finite score can never make the warp pick an index
+// twice or out of range.
+__device__ __forceinline__ void topk_warp(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
+                                          float routed_scale, int32_t* idx_row, float* w_row)
+{
+    const int lane = threadIdx.x & 31;
+    constexpr int kPer = kMaxExperts / 32;
+    float s[kPer], c[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            const float l = lrow[e];
+            s[i] = 1.0f / (1.0f + expf(-l));
+            const float ci = s[i] + sel_bias[e];
+            c[i] = (ci == ci) ? ci : -INFINITY;  // NaN ranks last: keeps the order total
+        } else {
+            s[i] = 0.f;
+            c[i] = 0.f;
+        }
+    }
+    uint32_t taken = 0;
+    int my_idx = 0;
+    float my_s = 0.f;
+    for (int j = 0; j < k; ++j) {
+        float bv = 0.f;
+        int bi = -1;
+        float bs = 0.f;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && (bi < 0 || c[i] > bv)) {
+                bv = c[i];
+                bi = e;
+                bs = s[i];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+            const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
+            if (oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oi < bi))) {
+                bv = ov;
+                bi = oi;
+                bs = os;
+            }
+        }
+        if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
+        if (lane == j) {
+            my_idx = bi;
+            my_s = bs;
+        }
+    }
+    float total = 0.f;
+    for (int j = 0; j < k; ++j) total += __shfl_sync(0xFFFFFFFFu, my_s, j);
+    if (lane < k) {
+        idx_row[lane] = my_idx;
+        w_row[lane] = routed_scale * my_s / total;
+    }
+}
+
+// One warp per token, logits from global memory (layer path).
+__global__ void __launch_bounds__(256)
+router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                   const float* __restrict__ sel_bias, float routed_scale,
+                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w)
+{
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;  // whole warp leaves together
+    topk_warp(logits + (size_t)t * E, E, k, sel_bias, routed_scale, topk_idx + (size_t)t * k,
+              topk_w + (size_t)t * k);
+}
+
+// Scratch-free router for the stand-alone entry point.  A cluster of
+// kRouterCluster CTAs owns kRouterTokens tokens; CTA r scores experts
+// e = r, r + kRouterCluster, ... (one warp per expert row, lanes split H) and
+// writes the logits into CTA 0's shared memory through distributed shared
+// memory; after a cluster barrier CTA 0 takes the top-k, one warp per token.
+constexpr int kRouterCluster = 8;
+constexpr int kRouterClusterThreads = 512;
+
+template <bool kBf16>
+__global__ void __cluster_dims__(kRouterCluster, 1, 1) __launch_bounds__(kRouterClusterThreads)
+router_cluster_kernel(const void* __restrict__ x, int T, int H, const float* __restrict__ w_router,
+                      const float* __restrict__ sel_bias, int E, int k, float routed_scale,
+                      int32_t* __restrict__ topk_idx, float* __restrict__ topk_w)
+{
+    __shared__ float s_logits[kRouterTokens][kMaxExperts];
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int t0 = (blockIdx.x / kRouterCluster) * kRouterTokens;
+    const int nt = min(kRouterTokens, T - t0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kWarps = kRouterClusterThreads / 32;
+    float* dst = cluster.map_shared_rank(&s_logits[0][0], 0);
+    const size_t xrow_bytes = (size_t)H * (kBf16 ? 2 : 4);
+    const char* xb = static_cast<const char*>(x) + (size_t)t0 * xrow_bytes;
+
+    for (int e = rank + kRouterCluster * warp; e < E; e += kRouterCluster * kWarps) {
+        const float* wrow = w_router + (size_t)e * H;
+        float acc[kRouterTokens];
+#pragma unroll
+        for (int t = 0; t < kRouterTokens; ++t) acc[t] = 0.f;
+        for (int i = lane * 4; i < H; i += 32 * 4) {
+            const float4 wv = *reinterpret_cast<const float4*>(wrow + i);
+#pragma unroll
+            for (int t = 0; t < kRouterTokens; ++t) {
+                if (t < nt) {
+                    const float4 v = load_act4<kBf16>(xb + t * xrow_bytes, i);
+                    acc[t] = fmaf(wv.x, v.x, acc[t]);
+                    acc[t] = fmaf(wv.y, v.y, acc[t]);
+                    acc[t] = fmaf(wv.z, v.z, acc[t]);
+                    acc[t] = fmaf(wv.w, v.w, acc[t]);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < kRouterTokens; ++t) {
+            const float v = warp_sum(acc[t]);
+            if (lane == 0 && t < nt) dst[t * kMaxExperts + e] = v;
+        }
+    }
+    cluster.sync();
+    if (rank == 0 && warp < nt)
+        topk_warp(&s_logits[warp][0], E, k, sel_bias, routed_scale, topk_idx + (size_t)(t0 + warp) * k,
+                  topk_w + (size_t)(t0 + warp) * k);
+}
+
+}  // namespace coli

@@ -1,0 +1,130 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel launched).
+
+The library loads, exports every function include/coli.h declares, and rejects
+bad arguments on the host before touching CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def coli():
+    from int4_routed_expert_bias_b200 import _build
+    _build.build()
+    import int4_routed_expert_bias_b200 as m
+    return m
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"COLI_API\s+[\w\s\*]+?\b(coli_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("coli_router_topk", "coli_expert_union", "coli_moe_workspace_size", "coli_moe_forward",
+              "coli_status_string", "coli_last_error", "coli_moe_profile_next"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(coli):
+    lib = coli.lib()
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(coli):
+    assert coli.status_string(0) == "COLI_OK"
+    assert coli.status_string(3) == "COLI_ERR_WORKSPACE"
+    assert coli.status_string(99) == "COLI_ERR_UNKNOWN"
+
+
+def _layer(coli, **over):
+    fake = 1 << 20  # non-null, aligned host integers: never dereferenced by argument checks
+    kw = dict(hidden=6144, ffn=2048, n_experts=256, top_k=8, group=64, routed_scale=2.5,
+              w_router=fake, sel_bias=fake, gate_q=fake, up_q=fake, down_q=fake,
+              gate_s=fake, up_s=fake, down_s=fake)
+    kw.update(over)
+    s = coli._LayerStruct()
+    for k, v in kw.items():
+        setattr(s, k, v)
+    return s
+
+
+def _fwd(coli, s, T=1, x=1 << 20, out=1 << 20, ws=1 << 20, ws_bytes=1 << 40, xt=0, ot=0):
+    return coli.lib().coli_moe_forward(ctypes.byref(s), x, xt, T, out, ot, ws, ws_bytes, None, None, None)
+
+
+def test_workspace_size_is_positive_and_grows(coli):
+    s = _layer(coli)
+    w1 = coli.lib().coli_moe_workspace_size(ctypes.byref(s), 1)
+    w64 = coli.lib().coli_moe_workspace_size(ctypes.byref(s), 64)
+    assert 0 < w1 < w64
+    assert coli.lib().coli_moe_workspace_size(None, 1) == 0
+    assert coli.lib().coli_moe_workspace_size(ctypes.byref(_layer(coli, hidden=100)), 1) == 0
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(hidden=100), 1), (dict(hidden=0), 1), (dict(ffn=96), 1), (dict(top_k=0), 1),
+    (dict(top_k=33), 1), (dict(n_experts=4, top_k=8), 1), (dict(n_experts=2000), 1),
+    (dict(group=128), 2), (dict(hidden=32768), 2), (dict(w_router=0), 1), (dict(gate_q=(1 << 20) + 8), 1),
+    (dict(routed_scale=float("inf")), 1),
+])
+def test_forward_rejects_bad_layers(coli, over, status):
+    assert _fwd(coli, _layer(coli, **over)) == status
+    assert coli.last_error() != ""
+
+
+def test_forward_rejects_bad_calls(coli):
+    s = _layer(coli)
+    assert _fwd(coli, s, T=-1) == 1
+    assert _fwd(coli, s, T=70000) == 1
+    assert _fwd(coli, s, xt=7) == 1
+    assert _fwd(coli, s, ot=7) == 1
+    assert _fwd(coli, s, x=0) == 1
+    assert _fwd(coli, s, x=(1 << 20) + 4) == 1
+    assert _fwd(coli, s, ws=(1 << 20) + 16) == 1
+    need = coli.lib().coli_moe_workspace_size(ctypes.byref(s), 1)
+    assert _fwd(coli, s, ws_bytes=need - 1) == 3
+    assert "workspace" in coli.last_error()
+
+
+def test_empty_forward_is_ok_without_launching(coli):
+    assert _fwd(coli, _layer(coli), T=0, x=0, out=0, ws=0, ws_bytes=0) == 0
+
+
+def test_router_rejects_bad_calls(coli):
+    L = coli.lib()
+    fake = 1 << 20
+    assert L.coli_router_topk(fake, 0, 1, 100, fake, fake, 256, 8, 2.5, fake, fake, None) == 1
+    assert L.coli_router_topk(fake, 0, 1, 6144, fake, fake, 4, 8, 2.5, fake, fake, None) == 1
+    assert L.coli_router_topk(fake, 3, 1, 6144, fake, fake, 256, 8, 2.5, fake, fake, None) == 1
+    assert L.coli_router_topk(None, 0, 1, 6144, fake, fake, 256, 8, 2.5, fake, fake, None) == 1
+    assert L.coli_router_topk(fake + 4, 0, 1, 6144, fake, fake, 256, 8, 2.5, fake, fake, None) == 1
+    assert L.coli_router_topk(fake, 0, 1, 6144, fake, fake, 256, 8, float("nan"), fake, fake, None) == 1
+    assert L.coli_router_topk(None, 0, 0, 6144, None, None, 256, 8, 2.5, None, None, None) == 0
+
+
+def test_union_rejects_bad_calls(coli):
+    L = coli.lib()
+    fake = 1 << 20
+    assert L.coli_expert_union(fake, -1, 8, 256, fake, fake, fake, fake, fake, fake, None) == 1
+    assert L.coli_expert_union(fake, 1, 0, 256, fake, fake, fake, fake, fake, fake, None) == 1
+    assert L.coli_expert_union(fake, 1, 8, 4, fake, fake, fake, fake, fake, fake, None) == 1
+    assert L.coli_expert_union(fake, 1, 8, 256, None, fake, fake, fake, fake, fake, None) == 1
+    assert L.coli_expert_union(None, 1, 8, 256, fake, fake, fake, fake, fake, fake, None) == 1
+
+
+def test_profile_hook_arms_and_disarms(coli):
+    L = coli.lib()
+    assert L.coli_moe_profile_next(None, 0) == 0
+    assert L.coli_moe_profile_next(1 << 20, -1) == 1

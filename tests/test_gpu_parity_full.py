@@ -1,0 +1,93 @@
+"""GPU parity at the full layer shape (H 6144, F 2048, 256 routed experts + 1
+shared, top-8), through the same entry point and launch path the benchmark
+times, for the four full-size workloads (decode-1, verify-4, decode-64,
+prefill-4096).
+
+Routing and the union are compared for every token; the layer output for every
+token of the small batches and for sampled tokens of the large ones (the
+oracle computes tokens independently: a T-token call equals T one-token calls).
+"""
+import numpy as np
+import pytest
+
+import inputs
+import oracle
+import _support as S
+
+pytestmark = pytest.mark.gpu
+
+SEED = 20261202
+LAYER = 0
+
+
+@pytest.fixture(scope="module")
+def full():
+    import torch
+    import int4_routed_expert_bias_b200 as coli
+    c = inputs.CONFIGS[1]
+    bufs = S.device_layer_generated(coli, torch, c, SEED, LAYER)
+    torch.cuda.synchronize()
+    cache = {}
+
+    def host_expert(e):
+        if e not in cache:
+            cache[e] = inputs.gen_expert_host(c, SEED, LAYER, e)
+        return cache[e]
+
+    yield coli, torch, bufs, host_expert
+    del bufs
+    torch.cuda.empty_cache()
+
+
+def _layer(coli, torch, c, bufs, w_router, sel_bias):
+    return coli.Layer(c.H, c.F, c.E, c.k, c.routed_scale, torch.from_numpy(w_router).cuda(),
+                      torch.from_numpy(sel_bias).cuda(), bufs["gate_q"], bufs["gate_s"], bufs["up_q"],
+                      bufs["up_s"], bufs["down_q"], bufs["down_s"])
+
+
+def test_device_generator_matches_host(full):
+    coli, torch, bufs, host_expert = full
+    for e in (0, 17, 256):
+        h = host_expert(e)
+        for n in ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s"):
+            assert np.array_equal(bufs[n][e].cpu().numpy(), h[n]), (e, n)
+
+
+@pytest.mark.parametrize("cfg,n_sample", [(1, 1), (2, 4), (3, 6), (4, 5)])
+def test_full_size_layer_matches_oracle(full, cfg, n_sample):
+    coli, torch, bufs, host_expert = full
+    c = inputs.CONFIGS[cfg]
+    w_router, sel_bias = inputs.router_params(c, SEED, LAYER)
+    x, _ = S.x_without_ties(c, SEED, 0, LAYER, w_router, sel_bias)
+    L = _layer(coli, torch, c, bufs, w_router, sel_bias)
+    T = c.T
+    xd = S.to_device_x(x, torch)
+    out = torch.empty((T, c.H), dtype=torch.bfloat16 if c.out_dtype == "bf16" else torch.float32,
+                      device="cuda")
+    ws = torch.empty(coli.moe_workspace_size(L, T), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((T, c.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, c.k), dtype=torch.float32, device="cuda")
+    coli.moe_forward(L, xd, out, ws, idx, w)
+    torch.cuda.synchronize()
+    idx, w = idx.cpu().numpy(), w.cpu().numpy()
+    out = S.output_to_f64(out, torch)
+
+    # routing and union: every token, bit-exact
+    ridx, rw = oracle.route(x, w_router, sel_bias, c.k, c.routed_scale)
+    assert np.array_equal(idx, ridx)
+    np.testing.assert_allclose(w, rw, rtol=2e-6)
+    u = oracle.union(ridx, c.E)
+    if cfg == 2:
+        assert 8 <= u["n_active"] <= 32
+    if cfg == 3:
+        assert u["count"].max() > 8  # the Zipf bias makes hot experts
+
+    # outputs: sampled tokens against the oracle layer
+    rng = np.random.default_rng(cfg)
+    tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, n_sample), replace=False)]))[:max(n_sample, 1)]
+    need = set(ridx[tokens].ravel().tolist()) | {c.E}
+    experts = {e: host_expert(e) for e in need}
+    _, _, rout = oracle.moe_layer(x[tokens], c.H, c.F, c.E, c.k, c.routed_scale, w_router, sel_bias, experts)
+    tol = 1e-2 if c.out_dtype == "bf16" else S.TOL_DECODE
+    err = S.rel_inf_err(out[tokens], rout)
+    assert err <= tol, (cfg, err)
