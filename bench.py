@@ -29,7 +29,7 @@ import inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (% roofline) at batch 1/4/64/4096"
 SEED = 1234
-N_LAYERS = 8
+N_LAYERS = 8  # resident layers cycled (bench --layers overrides it for profiling runs)
 STAGE_NAMES = ("route", "union", "gateup", "down", "combine")
 # our kernels per layer call on the current path (router scores, top-k, union,
 # gate/up, down, combine)
@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--config", type=int, default=1, choices=[1, 2, 3, 4])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=8, help="resident layers cycled (profiling: fewer)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="routed experts per layer (0 = the workload's; profiling: fewer, same per-call bytes)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
@@ -253,7 +256,12 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     import int4_routed_expert_bias_b200 as coli
 
+    global N_LAYERS
+    N_LAYERS = args.layers
     c = inputs.CONFIGS[args.config]
+    if args.experts:
+        c = inputs.Config(c.cfg, f"{c.name}-E{args.experts}", c.H, c.F, args.experts, c.k, c.T, c.x_dtype,
+                          c.out_dtype, args.layers)
     seed = SEED + 1000 * rank
     hbm_peak, _, peak_kind = measured_peaks()
 

@@ -34,16 +34,30 @@ router_logits_kernel(const void* __restrict__ x, int T, int H, const float* __re
 #pragma unroll
     for (int t = 0; t < kRouterTokens; ++t) acc[t] = 0.f;
 
-    for (int i = threadIdx.x * 4; i < H; i += kRouterThreads * 4) {
-        const float4 w = *reinterpret_cast<const float4*>(wrow + i);
+    // Issue every weight load of a pass before the first FMA: up to kUnroll
+    // 16-byte loads in flight per thread (H = 6144 needs 6).
+    constexpr int kUnroll = 8;
+    for (int base = threadIdx.x * 4; base < H; base += kUnroll * kRouterThreads * 4) {
+        float4 wv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = base + u * kRouterThreads * 4;
+            wv[u] = i < H ? *reinterpret_cast<const float4*>(wrow + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
         for (int t = 0; t < kRouterTokens; ++t) {
             if (t < nt) {
-                const float4 v = load_act4<kBf16>(xb + t * xrow_bytes, i);
-                acc[t] = fmaf(w.x, v.x, acc[t]);
-                acc[t] = fmaf(w.y, v.y, acc[t]);
-                acc[t] = fmaf(w.z, v.z, acc[t]);
-                acc[t] = fmaf(w.w, v.w, acc[t]);
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int i = base + u * kRouterThreads * 4;
+                    if (i < H) {
+                        const float4 v = load_act4<kBf16>(xb + t * xrow_bytes, i);
+                        acc[t] = fmaf(wv[u].x, v.x, acc[t]);
+                        acc[t] = fmaf(wv[u].y, v.y, acc[t]);
+                        acc[t] = fmaf(wv[u].z, v.z, acc[t]);
+                        acc[t] = fmaf(wv[u].w, v.w, acc[t]);
+                    }
+                }
             }
         }
     }

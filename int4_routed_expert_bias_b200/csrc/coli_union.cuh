@@ -103,7 +103,7 @@ union_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
 
     // stable scatter
     for (int base = 0; base < P; base += kUnionThreads) {
-        for (int i = tid; i < kUnionWarps * E; i += kUnionThreads) (&s_wcnt[0][0])[i] = 0;
+        for (int i = tid; i < kUnionWarps * E; i += kUnionThreads) s_wcnt[i / E][i % E] = 0;
         __syncthreads();
         const int p = base + tid;
         int e = p < P ? topk_idx[p] : -1;
