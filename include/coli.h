@@ -155,6 +155,40 @@ enum {
  */
 COLI_API coli_status coli_moe_profile_next(cudaEvent_t* events, int n_events);
 
+/*
+ * Allocation-free variant of coli_moe_forward (the colibri pages have no
+ * counterpart: it exists for callers of this library, not for the method).
+ *
+ * Some callers cannot hand the library a workspace.  cudaMalloc and cudaFree
+ * synchronise the whole device, so a latency-bound decode loop that must not
+ * stall the GPU cannot call them between tokens; and a library embedded in a
+ * host framework that owns every device allocation (its own pool, its own
+ * accounting) may not be allowed to allocate on its own at all.  This entry
+ * point takes the same arguments as coli_moe_forward minus the workspace and
+ * uses instead a scratch array compiled into libcoli.so as a file-scope
+ * __device__ array of COLI_NOALLOC_SCRATCH_BYTES bytes.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Limits and behaviour:
+ *   - A batch is accepted when coli_moe_workspace_size(layer, T) is at most
+ *     COLI_NOALLOC_SCRATCH_BYTES (8 MiB: up to 28 tokens at hidden 6144, ffn
+ *     2048, 256 experts, top-8); larger batches return COLI_ERR_WORKSPACE
+ *     with the sizes in coli_last_error() and launch nothing.
+ *   - Every GPU that loads the library holds the 8 MiB array until the process
+ *     exits.  The first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that first
+ *     call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (nothing in it needs to start at zero: every call writes what it
+ *     reads).  Calls whose work may overlap on the GPU (different streams, or
+ *     different host threads without ordering) race on it and give wrong
+ *     results; order them on one stream.
+ */
+#define COLI_NOALLOC_SCRATCH_BYTES (8u << 20)
+COLI_API coli_status coli_moe_forward_noalloc(const coli_moe_layer* layer, const void* x, coli_dtype xt,
+                                              int T, void* out, coli_dtype ot, int32_t* topk_idx_out,
+                                              float* topk_w_out, cudaStream_t stream);
+
 COLI_API const char* coli_status_string(coli_status status);
 COLI_API const char* coli_last_error(void);
 

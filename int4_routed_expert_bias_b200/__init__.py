@@ -32,6 +32,8 @@ _lib.coli_moe_workspace_size.restype = ctypes.c_size_t
 _lib.coli_moe_workspace_size.argtypes = [_p, _i]
 _lib.coli_moe_forward.restype = _i
 _lib.coli_moe_forward.argtypes = [_p, _p, _i, _i, _p, _i, _p, ctypes.c_size_t, _p, _p, _p]
+_lib.coli_moe_forward_noalloc.restype = _i
+_lib.coli_moe_forward_noalloc.argtypes = [_p, _p, _i, _i, _p, _i, _p, _p, _p]
 _lib.coli_moe_profile_next.restype = _i
 _lib.coli_moe_profile_next.argtypes = [_p, _i]
 _lib.coli_status_string.restype = ctypes.c_char_p
@@ -132,6 +134,14 @@ def moe_forward(layer, x, out, workspace, topk_idx_out=None, topk_w_out=None, st
     _check(_lib.coli_moe_forward(layer.ref, _ptr(x), _dtype_code(x), T, _ptr(out), _dtype_code(out),
                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _ptr(topk_idx_out), _ptr(topk_w_out), _stream(stream)))
+
+
+def moe_forward_noalloc(layer, x, out, topk_idx_out=None, topk_w_out=None, stream=None):
+    """moe_forward without a caller workspace: the library's static per-device
+    scratch (COLI_NOALLOC_SCRATCH_BYTES) is used instead; see include/coli.h."""
+    _check(_lib.coli_moe_forward_noalloc(layer.ref, _ptr(x), _dtype_code(x), x.shape[0], _ptr(out),
+                                         _dtype_code(out), _ptr(topk_idx_out), _ptr(topk_w_out),
+                                         _stream(stream)))
 
 
 def moe_profile_next(events):

@@ -379,3 +379,55 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of coli_moe_forward: the workspace is a file-scope
+// __device__ array compiled into the library (COLI_NOALLOC_SCRATCH_BYTES per
+// device, resident until the process exits), for callers that cannot allocate
+// device memory themselves.  Host code never passes the array's name to a
+// kernel (on the host it names a host-side stand-in); it passes the device
+// address looked up once per device with cudaGetSymbolAddress.
+
+namespace {
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[COLI_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on the
+// first call per device, with that device current).
+coli_status noalloc_scratch(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(COLI_ERR_UNSUPPORTED, "device %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return COLI_OK;
+}
+
+}  // namespace
+
+extern "C" coli_status coli_moe_forward_noalloc(const coli_moe_layer* L, const void* x, coli_dtype xt, int T,
+                                                void* out, coli_dtype ot, int32_t* topk_idx_out,
+                                                float* topk_w_out, cudaStream_t stream)
+{
+    const size_t need = coli_moe_workspace_size(L, T);  // 0 for an invalid layer: forward reports why
+    if (need > (size_t)COLI_NOALLOC_SCRATCH_BYTES)
+        return fail(COLI_ERR_WORKSPACE,
+                    "T=%d needs %zu bytes of scratch; the static scratch holds %zu bytes (use coli_moe_forward)",
+                    T, need, (size_t)COLI_NOALLOC_SCRATCH_BYTES);
+    void* ws = nullptr;
+    coli_status st = noalloc_scratch(&ws);
+    if (st != COLI_OK) return st;
+    return coli_moe_forward(L, x, xt, T, out, ot, ws, (size_t)COLI_NOALLOC_SCRATCH_BYTES, topk_idx_out,
+                            topk_w_out, stream);
+}
