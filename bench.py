@@ -31,9 +31,15 @@ METRIC = "MoE-layer tokens/s and achieved HBM GB/s (% roofline) at batch 1/4/64/
 SEED = 1234
 N_LAYERS = 8  # resident layers cycled (bench --layers overrides it for profiling runs)
 STAGE_NAMES = ("route", "union", "gateup", "down", "combine")
-# our kernels per layer call on the current path (router scores, top-k, union,
-# gate/up, down, combine)
-KERNELS_PER_CALL = 6
+
+
+def kernels_per_call(T, E):
+    """Our kernel launches in one layer call: batch 1 runs router scores, gate/up
+    (with top-k), down and combine; larger batches run router scores, top-k +
+    union (one kernel up to 256 tokens), gate/up, down and combine."""
+    if T == 1:
+        return 4
+    return 5 if (T <= 256 and E <= 256) else 6
 
 
 def parse():
@@ -371,11 +377,12 @@ def run_ours(args):
                                           "layer_gbs": layer_gbs,
                                           "layer_frac_of_hbm_peak": layer_gbs / hbm_peak,
                                           "stage_ms": stage_ms}),
-            "roofline": {"kernel": "expert_phase_kernel<gateup> (gate/up + SwiGLU, routed and shared)",
+            "roofline": {"kernel": ("gateup_single_kernel" if c.T == 1 else "expert_phase_kernel<gateup>")
+                         + " (gate/up + SwiGLU, routed and shared experts)",
                          "bound": "hbm", "achieved": gu_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": gu_gbs / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
                          "alg_bytes_per_launch": gu_alg},
-            "gpu_launches": steps * KERNELS_PER_CALL,
+            "gpu_launches": steps * kernels_per_call(c.T, c.E),
             "clocks": clocks}
 
     # end to end through the public call with host buffers: pinned x in, out back

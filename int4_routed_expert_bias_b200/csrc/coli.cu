@@ -14,6 +14,7 @@
 #include "coli.h"
 #include "coli_common.cuh"
 #include "coli_decode.cuh"
+#include "coli_decode1.cuh"
 #include "coli_router.cuh"
 #include "coli_union.cuh"
 
@@ -91,7 +92,10 @@ coli_status device_info(DeviceInfo** out)
             (e = allow_smem(expert_phase_kernel<true, true, 1>, lim)) != cudaSuccess ||
             (e = allow_smem(expert_phase_kernel<true, true, 4>, lim)) != cudaSuccess ||
             (e = allow_smem(expert_phase_kernel<false, false, 1>, lim)) != cudaSuccess ||
-            (e = allow_smem(expert_phase_kernel<false, false, 4>, lim)) != cudaSuccess)
+            (e = allow_smem(expert_phase_kernel<false, false, 4>, lim)) != cudaSuccess ||
+            (e = allow_smem(gateup_single_kernel<false>, lim)) != cudaSuccess ||
+            (e = allow_smem(gateup_single_kernel<true>, lim)) != cudaSuccess ||
+            (e = allow_smem(down_single_kernel<0>, lim)) != cudaSuccess)
             return cuda_fail(e, "kernel attribute setup");
         d.smem_optin = lim;
         d.ready = true;
@@ -102,10 +106,10 @@ coli_status device_info(DeviceInfo** out)
 
 // Resident blocks per SM for the actual dynamic smem of one launch.
 template <typename Kern>
-int blocks_per_sm(Kern k, size_t smem)
+int blocks_per_sm(Kern k, size_t smem, int threads = kDecThreads)
 {
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kDecThreads, smem) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess) return 1;
     return occ > 0 ? occ : 1;
 }
 
@@ -204,19 +208,39 @@ struct StageTimer {
     }
 };
 
-coli_status launch_route(const void* x, coli_dtype xt, int T, int H, const float* w_router,
-                         const float* sel_bias, int E, int k, float routed_scale, float* logits,
-                         int32_t* idx, float* w, cudaStream_t s)
+coli_status launch_logits(const void* x, coli_dtype xt, int T, int H, const float* w_router, int E,
+                          float* logits, int32_t* zero_ctr, int n_zero, cudaStream_t s)
 {
     dim3 grid(E, (T + kRouterTokens - 1) / kRouterTokens);
-    if (xt == COLI_BF16) router_logits_kernel<true><<<grid, kRouterThreads, 0, s>>>(x, T, H, w_router, E, logits);
-    else router_logits_kernel<false><<<grid, kRouterThreads, 0, s>>>(x, T, H, w_router, E, logits);
-    const int warps_per_block = 8;
-    router_topk_kernel<<<(T + warps_per_block - 1) / warps_per_block, 256, 0, s>>>(
-        logits, T, E, k, sel_bias, routed_scale, idx, w);
+    if (xt == COLI_BF16)
+        router_logits_kernel<true><<<grid, kRouterThreads, 0, s>>>(x, T, H, w_router, E, logits, zero_ctr, n_zero);
+    else
+        router_logits_kernel<false><<<grid, kRouterThreads, 0, s>>>(x, T, H, w_router, E, logits, zero_ctr, n_zero);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? COLI_OK : cuda_fail(e, "router launch");
 }
+
+// Launch as a programmatic dependent of the previous kernel on the stream: its
+// launch may overlap the predecessor's tail; the kernel calls griddep_wait()
+// before it reads anything the predecessor wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// Batches up to this size take the top-k inside the union block.
+constexpr int kFusedTopkMaxT = 256;
 
 }  // namespace
 
@@ -276,8 +300,9 @@ coli_status coli_expert_union(const int32_t* topk_idx, int T, int k, int E, int3
     if (!count || !offset || !active || !n_active || (T > 0 && (!topk_idx || !perm || !inv_perm)))
         return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
     WorkLists wl{};
-    union_kernel<false><<<1, kUnionThreads, 0, stream>>>(topk_idx, T, k, E, count, offset, active,
-                                                         n_active, perm, inv_perm, wl);
+    TopkArgs tk{};
+    union_kernel<false, false><<<1, kUnionThreads, 0, stream>>>(const_cast<int32_t*>(topk_idx), T, k, E, count,
+                                                                offset, active, n_active, perm, inv_perm, wl, tk);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? COLI_OK : cuda_fail(e, "union launch");
 }
@@ -323,20 +348,70 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
 
     int32_t* idx = topk_idx_out ? topk_idx_out : w.idx;
     float* wt = topk_w_out ? topk_w_out : w.w;
-    const int TG = group_tokens(T, H, F, dev->smem_optin);
     const bool bf16 = (xt == COLI_BF16);
 
-    // Route
+    // One token: router scores, then gate/up (top-k in every CTA), then down with
+    // the combine fused; the union of a one-token batch is its k experts.
+    const size_t s1_gu = stage_smem_bytes(H, 1), s1_dn = stage_smem_bytes(F, k + 1);
+    // (batch-1 path: router scores, gate/up, down, combine; see coli_decode1.cuh)
+    if (T == 1 && E <= 256 && stage_geom(H).per_lane <= 2 * kHalf && stage_geom(F).per_lane <= 2 && H % 2 == 0 &&
+        s1_gu <= (size_t)dev->smem_optin && s1_dn <= (size_t)dev->smem_optin) {
+        if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
+        st = launch_logits(x, xt, 1, H, L->w_router, E, w.logits, nullptr, 0, stream);
+        if (st != COLI_OK) return st;
+        if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess ||
+            (e = tm.rec(COLI_STAGE_UNION, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_GATEUP, 0)) != cudaSuccess)
+            return cuda_fail(e, "event record");
+        SingleArgs sa{L->gate_q, L->gate_s, L->up_q, L->up_s, L->down_q, L->down_s, H, F, E, k,
+                      L->routed_scale, w.logits, L->sel_bias, x, idx, wt, w.h, w.partial, out};
+        {
+            auto kern = bf16 ? gateup_single_kernel<true> : gateup_single_kernel<false>;
+            if ((e = launch_pdl(kern, dev->sms * blocks_per_sm(kern, s1_gu, kSingleThreads), kSingleThreads, s1_gu,
+                                stream, sa)) != cudaSuccess)
+                return cuda_fail(e, "gate/up launch");
+        }
+        if ((e = tm.rec(COLI_STAGE_GATEUP, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_DOWN, 0)) != cudaSuccess)
+            return cuda_fail(e, "event record");
+        {
+            auto kern = down_single_kernel<0>;
+            if ((e = launch_pdl(kern, dev->sms * blocks_per_sm(kern, s1_dn, kSingleThreads), kSingleThreads, s1_dn,
+                                stream, sa)) != cudaSuccess)
+                return cuda_fail(e, "down launch");
+        }
+        if ((e = tm.rec(COLI_STAGE_DOWN, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_COMBINE, 0)) != cudaSuccess)
+            return cuda_fail(e, "event record");
+        {
+            const int blocks = (H / 4 + 127) / 128;
+            e = ot == COLI_BF16 ? launch_pdl(combine_single_kernel<true>, blocks, 128, 0, stream, w.partial, k + 1, H, out)
+                                : launch_pdl(combine_single_kernel<false>, blocks, 128, 0, stream, w.partial, k + 1, H, out);
+            if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+        }
+        if ((e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
+        e = cudaGetLastError();
+        return e == cudaSuccess ? COLI_OK : cuda_fail(e, "layer launch");
+    }
+
+    const int TG = group_tokens(T, H, F, dev->smem_optin);
+
+    // Route (router scores; the top-k runs in the union block for small batches)
     if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
-    st = launch_route(x, xt, T, H, L->w_router, L->sel_bias, E, k, L->routed_scale, w.logits, idx, wt, stream);
+    st = launch_logits(x, xt, T, H, L->w_router, E, w.logits, nullptr, 0, stream);
     if (st != COLI_OK) return st;
+    const bool fused_topk = T <= kFusedTopkMaxT && E <= 256;
+    if (!fused_topk)
+        router_topk_kernel<<<(T + 7) / 8, 256, 0, stream>>>(w.logits, T, E, k, L->sel_bias, L->routed_scale, idx, wt);
     if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
 
     // Union and work lists
     if ((e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess) return cuda_fail(e, "event record");
     WorkLists wl{w.pair_token, w.pair_w, w.ctl, w.g_expert, w.g_start, w.g_count, wt, TG};
-    union_kernel<true><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
-                                                        w.n_active, w.perm, w.inv_perm, wl);
+    TopkArgs tk{w.logits, L->sel_bias, L->routed_scale, wt};
+    if (fused_topk)
+        union_kernel<true, true><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
+                                                                  w.n_active, w.perm, w.inv_perm, wl, tk);
+    else
+        union_kernel<true, false><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
+                                                                   w.n_active, w.perm, w.inv_perm, wl, tk);
     if ((e = tm.rec(COLI_STAGE_UNION, 1)) != cudaSuccess) return cuda_fail(e, "event record");
 
     // Gate/up + SwiGLU for every token group (routed experts, then the shared expert)

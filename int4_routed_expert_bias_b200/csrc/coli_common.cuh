@@ -66,6 +66,13 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p)
 
 __device__ __forceinline__ float ldg_f32(const float* p) { return __ldg(p); }
 
+// Programmatic dependent launch: a kernel launched as a programmatic dependent
+// waits here until its predecessor grid has completed and flushed its writes
+// (a no-op when launched without the attribute); the predecessor may signal
+// early that dependents can start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __host__ __device__ __forceinline__ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace coli

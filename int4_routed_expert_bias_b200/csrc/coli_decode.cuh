@@ -13,7 +13,7 @@
 // shared memory, in fp32.
 #pragma once
 
-#include "coli_common.cuh"
+#include "coli_int4.cuh"
 
 namespace coli {
 
@@ -22,120 +22,12 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kGateUpRows = 2;   // rows per warp of each of gate and up
 constexpr int kDownRows = 4;     // rows per warp of down
 
-// Shared-memory image of TG activation vectors of length K, laid out so that
-// lane l reading chunk c = l + 32 i, float4 j finds it at ((i * 8 + j) * 32 + l):
-// conflict-free 16-byte loads.  m24[t][c] = -24 * (sum of the 32 values of chunk c).
-struct StageGeom {
-    int nch;       // chunks (32 values) per vector = K / 32
-    int per_lane;  // ceil(nch / 32)
-    int f4;        // float4 slots per vector = per_lane * 32 * 8
-};
-
-__host__ __device__ inline StageGeom stage_geom(int K)
-{
-    StageGeom g;
-    g.nch = K / kChunkK;
-    g.per_lane = (g.nch + 31) / 32;
-    g.f4 = g.per_lane * 32 * 8;
-    return g;
-}
-
-__host__ __device__ inline size_t stage_smem_bytes(int K, int TG)
-{
-    const StageGeom g = stage_geom(K);
-    return (size_t)TG * g.f4 * 16 + (size_t)TG * g.nch * 4;
-}
-
-// Stage n vectors (rows tok[0..n) of src, K values each, fp32 or bf16) into xs/m24.
-template <bool kBf16>
-__device__ __forceinline__ void stage_vectors(const void* __restrict__ src, size_t row_elems,
-                                              const int* tok, int n, const StageGeom& g,
-                                              float4* xs, float* m24)
-{
-    const int total = n * g.nch * 8;
-    const size_t esz = kBf16 ? 2 : 4;
-    for (int base = 0; base < total; base += blockDim.x) {
-        const int idx = base + threadIdx.x;
-        const bool valid = idx < total;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        int t = 0, c = 0, j = 0;
-        if (valid) {
-            t = idx / (g.nch * 8);
-            const int rem = idx - t * g.nch * 8;
-            c = rem >> 3;
-            j = rem & 7;
-            const char* row = static_cast<const char*>(src) + (size_t)tok[t] * row_elems * esz;
-            v = load_act4<kBf16>(row, c * kChunkK + j * 4);
-            xs[(size_t)t * g.f4 + ((c >> 5) * 8 + j) * 32 + (c & 31)] = v;
-        }
-        float part = (v.x + v.y) + (v.z + v.w);
-        part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
-        part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
-        part += __shfl_xor_sync(0xFFFFFFFFu, part, 4);
-        if (valid && j == 0) m24[t * g.nch + c] = -24.f * part;
-    }
-}
-
-template <int q>
-__device__ __forceinline__ uint32_t word_of(const uint4& w)
-{
-    if constexpr (q == 0) return w.x;
-    else if constexpr (q == 1) return w.y;
-    else if constexpr (q == 2) return w.z;
-    else return w.w;
-}
-
-// Accumulate, for NS row streams and up to TG staged vectors, the dot product of
-// one 16-byte chunk (32 nibbles, k = 32c..32c+31) with the vectors:
-//   sum_k q_k x_k = 16 * sum_k (1.5 + q_k/16) x_k - 24 * sum_k x_k,
-// then scale by the row's group scale.
-template <int NS, int TG>
-__device__ __forceinline__ void chunk_dot(const uint4 (&w)[NS], const float (&sc)[NS],
-                                          const float4* xs_i, int f4, const float* m24c, int nch,
-                                          int ntok, float (&acc)[NS][TG])
-{
-#pragma unroll
-    for (int t = 0; t < TG; ++t) {
-        if (t < ntok) {
-            float a[NS];
-#pragma unroll
-            for (int r = 0; r < NS; ++r) a[r] = 0.f;
-            const float4* xt = xs_i + (size_t)t * f4;
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const float4 xv = xt[jj * 32];
-#pragma unroll
-                for (int r = 0; r < NS; ++r) {
-                    uint32_t wd;
-                    if ((jj >> 1) == 0) wd = word_of<0>(w[r]);
-                    else if ((jj >> 1) == 1) wd = word_of<1>(w[r]);
-                    else if ((jj >> 1) == 2) wd = word_of<2>(w[r]);
-                    else wd = word_of<3>(w[r]);
-                    if (jj & 1) {
-                        a[r] = fmaf(nib_as_float<4>(wd), xv.x, a[r]);
-                        a[r] = fmaf(nib_as_float<5>(wd), xv.y, a[r]);
-                        a[r] = fmaf(nib_as_float<6>(wd), xv.z, a[r]);
-                        a[r] = fmaf(nib_as_float<7>(wd), xv.w, a[r]);
-                    } else {
-                        a[r] = fmaf(nib_as_float<0>(wd), xv.x, a[r]);
-                        a[r] = fmaf(nib_as_float<1>(wd), xv.y, a[r]);
-                        a[r] = fmaf(nib_as_float<2>(wd), xv.z, a[r]);
-                        a[r] = fmaf(nib_as_float<3>(wd), xv.w, a[r]);
-                    }
-                }
-            }
-            const float m = m24c[t * nch];
-#pragma unroll
-            for (int r = 0; r < NS; ++r) acc[r][t] = fmaf(sc[r], fmaf(a[r], 16.f, m), acc[r][t]);
-        }
-    }
-}
-
 // Dot products of NS int4 rows (qrow[r]: packed bytes, srow[r]: scales) with
 // ntok staged vectors, reduced over the warp: every lane returns the totals.
+// The loads of the next chunk are issued before the current one is consumed.
 template <int NS, int TG>
 __device__ __forceinline__ void rows_dot(const uint8_t* const (&qrow)[NS], const float* const (&srow)[NS],
-                                         const StageGeom& g, const float4* xs, const float* m24,
+                                         const StageGeom& g, const float4* xs, const float* corr,
                                          int ntok, float (&acc)[NS][TG])
 {
     const int lane = threadIdx.x & 31;
@@ -162,15 +54,25 @@ __device__ __forceinline__ void rows_dot(const uint8_t* const (&qrow)[NS], const
 #pragma unroll 1
     for (int i = 0; i < g.per_lane; ++i, c += 32) {
         const int cn = c + 32;
-        if (cn < g.nch) {  // prefetch the next chunk while this one is consumed
+        if (cn < g.nch) {
 #pragma unroll
             for (int r = 0; r < NS; ++r) {
                 wn[r] = ldg_stream(qrow[r] + (size_t)cn * 16);
                 scn[r] = ldg_f32(srow[r] + (cn >> 1));
             }
         }
-        if (c < g.nch)
-            chunk_dot<NS, TG>(w, sc, xs + i * 256 + lane, g.f4, m24 + c, g.nch, ntok, acc);
+        if (c < g.nch) {
+#pragma unroll
+            for (int t = 0; t < TG; ++t) {
+                if (t < ntok) {
+                    float2 a[NS];
+                    chunk_acc_rows<NS>(w, xs + (size_t)t * g.f4 + i * 256, lane, a);
+                    const float cr = corr[t * g.nch + c];
+#pragma unroll
+                    for (int r = 0; r < NS; ++r) acc[r][t] = chunk_finish(a[r], cr, sc[r], acc[r][t]);
+                }
+            }
+        }
 #pragma unroll
         for (int r = 0; r < NS; ++r) {
             w[r] = wn[r];
@@ -213,7 +115,7 @@ expert_phase_kernel(PhaseArgs a)
     extern __shared__ __align__(16) unsigned char smem[];
     const StageGeom g = stage_geom(a.K);
     float4* xs = reinterpret_cast<float4*>(smem);
-    float* m24 = reinterpret_cast<float*>(smem + (size_t)TG * g.f4 * 16);
+    float* corr = reinterpret_cast<float*>(smem + (size_t)TG * g.f4 * 16);
     __shared__ int s_tok[TG];
     __shared__ int s_ntok;
     __shared__ int s_next;
@@ -245,8 +147,9 @@ expert_phase_kernel(PhaseArgs a)
         }
         if (!same) {  // uniform across the block
             __syncthreads();
-            if (kGateUp) stage_vectors<kBf16>(a.act, (size_t)a.K, tok, n, g, xs, m24);
-            else stage_vectors<false>(a.act, (size_t)a.K, tok, n, g, xs, m24);
+            auto rows = [&](int t) { return tok[t]; };
+            if (kGateUp) stage_vectors<kBf16>(a.act, a.K, n, rows, g, xs, corr);
+            else stage_vectors<false>(a.act, a.K, n, rows, g, xs, corr);
             if (threadIdx.x == 0) {
                 s_ntok = n;
 #pragma unroll
@@ -269,7 +172,7 @@ expert_phase_kernel(PhaseArgs a)
             }
         }
         float acc[NS][TG];
-        rows_dot<NS, TG>(qrow, srow, g, xs, m24, n, acc);
+        rows_dot<NS, TG>(qrow, srow, g, xs, corr, n, acc);
 
         // lane (r * TG + t) writes one result
 #pragma unroll

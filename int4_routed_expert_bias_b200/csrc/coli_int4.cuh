@@ -1,0 +1,153 @@
+// coli_int4.cuh -- int4-gs64 dot products on CUDA cores (decode path building blocks).
+//
+// Weights are stored as int4 with one fp32 scale per 64 along K ("gs64 build",
+// "colibri: 744B MoEをストレージから推論するCエンジン", section はじめにとソースが語らないこと);
+// decode keeps the arithmetic in fp32 ("Colibri 完全ガイド", section 詳細解説 step 3).
+//
+// Nibble -> float without an int->float conversion.  One shift of a packed
+// word w puts two neighbouring nibbles into two mantissa windows of 1.0f:
+//   window A, bits 19..22:  fa = 1 + (q_a + 8) / 16
+//   window B, bits 15..18:  fb = 1 + (q_b + 8) / 256
+// (the nibble's top bit is flipped, so q + 8 = nibble ^ 8 for two's complement).
+// Shifts w<<15, w<<7 and, with t = w>>12, t<<11, t<<3 place nibbles (1,0),
+// (3,2), (5,4), (7,6) into (A,B); each float is one lop3.  A packed fp32x2 FMA then takes one odd-k and
+// one even-k product.  Over a chunk of 32 k values:
+//   sum_k q_k x_k = 16 * sum_odd fa x + 256 * sum_even fb x
+//                   - 24 * sum_odd x - 264 * sum_even x,
+// the last two terms coming from the staged activations.  Window B keeps every
+// product exact to 2^-16 of |x|, far inside fp32-accumulate tolerances.
+#pragma once
+
+#include "coli_common.cuh"
+
+namespace coli {
+
+// (a & b) ^ c in one instruction
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ float2 nib_pair(uint32_t s)
+{
+    return make_float2(__uint_as_float(and_xor(s, 0x00780000u, 0x3FC00000u)),
+                       __uint_as_float(and_xor(s, 0x00078000u, 0x3F840000u)));
+}
+
+// Accumulate one packed word (k = 8q .. 8q+7 of a chunk) against activations
+// staged as swapped pairs: x01 = (x[8q+1], x[8q]), x23 = (x[8q+3], x[8q+2]), ...
+__device__ __forceinline__ float2 word_dot(uint32_t w, float4 xlo, float4 xhi, float2 acc)
+{
+    const uint32_t t = w >> 12;
+    acc = __ffma2_rn(nib_pair(w << 15), make_float2(xlo.x, xlo.y), acc);
+    acc = __ffma2_rn(nib_pair(w << 7), make_float2(xlo.z, xlo.w), acc);
+    acc = __ffma2_rn(nib_pair(t << 11), make_float2(xhi.x, xhi.y), acc);
+    acc = __ffma2_rn(nib_pair(t << 3), make_float2(xhi.z, xhi.w), acc);
+    return acc;
+}
+
+// total += scale * (sum_k q_k x_k) for one chunk, given its accumulators and the
+// chunk's correction corr = -24 * sum_odd x - 264 * sum_even x.
+__device__ __forceinline__ float chunk_finish(float2 acc, float corr, float scale, float total)
+{
+    return fmaf(scale, fmaf(acc.x, 16.f, fmaf(acc.y, 256.f, corr)), total);
+}
+
+// Per-lane accumulation of NS rows' chunks against one staged chunk; each x
+// slot is loaded once and used for every row.  xrow = the staged vector's
+// float4 row block of this lane's chunk (xs + i * 256), slot j at
+// xrow[j * 32 + (lane ^ j)].
+template <int NS>
+__device__ __forceinline__ void chunk_acc_rows(const uint4 (&w)[NS], const float4* xrow, int lane,
+                                               float2 (&acc)[NS])
+{
+#pragma unroll
+    for (int r = 0; r < NS; ++r) acc[r] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 xlo = xrow[(2 * q) * 32 + (lane ^ (2 * q))];
+        const float4 xhi = xrow[(2 * q + 1) * 32 + (lane ^ (2 * q + 1))];
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {
+            const uint32_t wd = q == 0 ? w[r].x : q == 1 ? w[r].y : q == 2 ? w[r].z : w[r].w;
+            acc[r] = word_dot(wd, xlo, xhi, acc[r]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Staging of activation vectors in shared memory.
+//
+// One vector of K values becomes K/4 float4 slots: chunk c (32 values), slot
+// j (values 4j..4j+3 of the chunk) lives at ((c / 32) * 8 + j) * 32 + ((c % 32) ^ j).
+// Lane l reading chunk c = l + 32 i, slot j touches 32 distinct 16-byte words of
+// one 512-byte row, and the staging threads (8 consecutive threads per chunk,
+// one per slot) write distinct banks: both directions are conflict-free.
+// Each slot holds the swapped pairs (x1, x0, x3, x2).
+// corr[c] = -24 * (odd-k sum) - 264 * (even-k sum) of chunk c.
+
+struct StageGeom {
+    int nch;       // chunks per vector = K / 32
+    int per_lane;  // ceil(nch / 32)
+    int f4;        // float4 slots per vector = per_lane * 256
+};
+
+__host__ __device__ inline StageGeom stage_geom(int K)
+{
+    StageGeom g;
+    g.nch = K / kChunkK;
+    g.per_lane = (g.nch + 31) / 32;
+    g.f4 = g.per_lane * 256;
+    return g;
+}
+
+__host__ __device__ inline size_t stage_smem_bytes(int K, int n_vectors)
+{
+    const StageGeom g = stage_geom(K);
+    return (size_t)n_vectors * g.f4 * 16 + (size_t)n_vectors * g.nch * 4;
+}
+
+// Stage n vectors; load(t, i) returns values i..i+3 of vector t (fp32).
+// All threads of the block call this (it uses warp shuffles).
+template <typename Load4>
+__device__ __forceinline__ void stage_vectors_fn(int n, Load4 load, const StageGeom& g, float4* xs, float* corr)
+{
+    const int total = n * g.nch * 8;
+    for (int base = 0; base < total; base += blockDim.x) {
+        const int idx = base + threadIdx.x;
+        const bool valid = idx < total;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        int t = 0, c = 0, j = 0;
+        if (valid) {
+            t = idx / (g.nch * 8);
+            const int rem = idx - t * g.nch * 8;
+            c = rem >> 3;
+            j = rem & 7;
+            v = load(t, c * kChunkK + j * 4);
+            xs[(size_t)t * g.f4 + ((c >> 5) * 8 + j) * 32 + ((c & 31) ^ j)] = make_float4(v.y, v.x, v.w, v.z);
+        }
+        float odd = v.y + v.w, even = v.x + v.z;
+        odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 1);
+        even += __shfl_xor_sync(0xFFFFFFFFu, even, 1);
+        odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 2);
+        even += __shfl_xor_sync(0xFFFFFFFFu, even, 2);
+        odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 4);
+        even += __shfl_xor_sync(0xFFFFFFFFu, even, 4);
+        if (valid && j == 0) corr[t * g.nch + c] = fmaf(-24.f, odd, -264.f * even);
+    }
+}
+
+// Stage n vectors; vector v is row rows(v) of src (K values each, fp32 or bf16).
+template <bool kBf16, typename RowOf>
+__device__ __forceinline__ void stage_vectors(const void* __restrict__ src, int K, int n, RowOf rows,
+                                              const StageGeom& g, float4* xs, float* corr)
+{
+    const size_t row_bytes = (size_t)K * (kBf16 ? 2 : 4);
+    stage_vectors_fn(n, [&](int t, int i) {
+        return load_act4<kBf16>(static_cast<const char*>(src) + (size_t)rows(t) * row_bytes, i);
+    }, g, xs, corr);
+}
+
+}  // namespace coli

@@ -15,14 +15,16 @@ constexpr int kRouterTokens = 4;     // tokens per router block
 constexpr int kRouterThreads = 256;
 
 // logits[t, e] for one expert row e (blockIdx.x) and up to kRouterTokens tokens
-// (blockIdx.y).  The row of w_router is read once per token group with 16-byte
+// (blockIdx.y); optionally zeroes n_zero counters used by the next kernels.  The row of w_router is read once per token group with 16-byte
 // loads; the per-thread partial sums are reduced in a fixed order, so the
 // result is deterministic.
 template <bool kBf16>
 __global__ void __launch_bounds__(kRouterThreads)
 router_logits_kernel(const void* __restrict__ x, int T, int H, const float* __restrict__ w_router,
-                     int E, float* __restrict__ logits)
+                     int E, float* __restrict__ logits, int32_t* __restrict__ zero_ctr, int n_zero)
 {
+    if (zero_ctr && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_ctr[i] = 0;
     const int e = blockIdx.x;
     const int t0 = blockIdx.y * kRouterTokens;
     const int nt = min(kRouterTokens, T - t0);
@@ -81,11 +83,12 @@ router_logits_kernel(const void* __restrict__ x, int T, int H, const float* __re
 // renormalised weights.  Lane j keeps the j-th selection.  The arg-max key is
 // (c desc, index asc); a non-finite score can never make the warp pick an index
 // twice or out of range.
-__device__ __forceinline__ void topk_warp(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
-                                          float routed_scale, int32_t* idx_row, float* w_row)
+// kPer = experts held per lane (E <= 32 * kPer).
+template <int kPer>
+__device__ __forceinline__ void topk_warp_t(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
+                                            float routed_scale, int32_t* idx_row, float* w_row)
 {
     const int lane = threadIdx.x & 31;
-    constexpr int kPer = kMaxExperts / 32;
     float s[kPer], c[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
@@ -139,6 +142,13 @@ __device__ __forceinline__ void topk_warp(const float* lrow, int E, int k, const
         idx_row[lane] = my_idx;
         w_row[lane] = routed_scale * my_s / total;
     }
+}
+
+__device__ __forceinline__ void topk_warp(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
+                                          float routed_scale, int32_t* idx_row, float* w_row)
+{
+    if (E <= 256) topk_warp_t<8>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
+    else topk_warp_t<kMaxExperts / 32>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
 }
 
 // One warp per token, logits from global memory (layer path).

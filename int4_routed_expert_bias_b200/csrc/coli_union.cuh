@@ -6,6 +6,7 @@
 #pragma once
 
 #include "coli_common.cuh"
+#include "coli_router.cuh"
 
 namespace coli {
 
@@ -22,6 +23,15 @@ struct WorkLists {
     int32_t* g_count;     // [G]: pairs in the group (<= group_tokens)
     const float* topk_w;  // [P]
     int group_tokens;     // tokens per group
+};
+
+// Optional fused top-k in front of the union (small batches): the router
+// scores are in logits [T, E]; topk_idx / topk_w receive the routing.
+struct TopkArgs {
+    const float* logits;
+    const float* sel_bias;
+    float routed_scale;
+    float* topk_w;
 };
 
 // Inclusive scan of one value per thread over the block (kUnionThreads threads).
@@ -55,13 +65,20 @@ __device__ __forceinline__ int block_incl_scan(int v, int* warp_tot)
 // inside a chunk a pair's rank among equal experts is its rank inside its warp
 // (match_any) plus the counts of that expert in earlier warps, so the order is
 // the stable (expert, p) order whatever the thread timing.
-template <bool kLists>
+template <bool kLists, bool kTopk>
 __global__ void __launch_bounds__(kUnionThreads)
-union_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
+union_kernel(int32_t* topk_idx, int T, int k, int E,
              int32_t* __restrict__ count, int32_t* __restrict__ offset,
              int32_t* __restrict__ active, int32_t* __restrict__ n_active,
-             int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, WorkLists wl)
+             int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, WorkLists wl, TopkArgs tk)
 {
+    if constexpr (kTopk) {
+        // Route first: one warp per token, written to topk_idx / topk_w
+        for (int t = threadIdx.x >> 5; t < T; t += kUnionWarps)
+            topk_warp_t<8>(tk.logits + (size_t)t * E, E, k, tk.sel_bias, tk.routed_scale,
+                           topk_idx + (size_t)t * k, tk.topk_w + (size_t)t * k);  // E <= 256 here
+        __syncthreads();
+    }
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_cursor[kMaxExperts];
     __shared__ uint8_t s_wcnt[kUnionWarps][kMaxExperts];
