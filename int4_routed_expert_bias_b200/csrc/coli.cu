@@ -354,7 +354,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     // the combine fused; the union of a one-token batch is its k experts.
     const size_t s1_gu = stage_smem_bytes(H, 1), s1_dn = stage_smem_bytes(F, k + 1);
     // (batch-1 path: router scores, gate/up, down, combine; see coli_decode1.cuh)
-    if (T == 1 && E <= 256 && stage_geom(H).per_lane <= 2 * kHalf && stage_geom(F).per_lane <= 2 && H % 2 == 0 &&
+    if (T == 1 && E <= 256 && H == 1024 * 2 * kHalf && F == 2048 &&
         s1_gu <= (size_t)dev->smem_optin && s1_dn <= (size_t)dev->smem_optin) {
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
         st = launch_logits(x, xt, 1, H, L->w_router, E, w.logits, nullptr, 0, stream);

@@ -43,77 +43,86 @@ struct SingleArgs {
     void* out;              // [H] fp32 or bf16
 };
 
-// Half of a gate/up unit's loads: chunks b0 .. b0+kHalf-1 (c = lane + 32 b) of
-// the gate row and of the up row.
+// Half of a gate/up unit: chunks c = lane + 32 b for b in [b0, b0 + kHalf) of the
+// gate row and of the up row (kPL chunks per lane in all).
 struct HalfRegs {
     uint4 w[kHalf][2];
     float sc[kHalf][2];
 };
 
-__device__ __forceinline__ void half_load(const SingleArgs& a, const StageGeom& g, int e, int n, int b0,
-                                          int lane, HalfRegs& r)
+template <int b0>
+__device__ __forceinline__ void half_load(const uint8_t* gq, const uint8_t* uq, const float* gs, const float* us,
+                                          HalfRegs& r)
 {
-    const size_t row = (size_t)e * a.F + n;
-    const uint8_t* gq = a.gate_q + row * ((size_t)a.H / 2);
-    const uint8_t* uq = a.up_q + row * ((size_t)a.H / 2);
-    const float* gs = a.gate_s + row * ((size_t)a.H / kGroup);
-    const float* us = a.up_s + row * ((size_t)a.H / kGroup);
+    // gq/uq point at this lane's first chunk (lane * 16), gs/us at the row's scales + lane / 2
 #pragma unroll
     for (int b = 0; b < kHalf; ++b) {
-        const int c = lane + 32 * (b0 + b);
-        if (b0 + b < g.per_lane && c < g.nch) {
-            r.w[b][0] = ldg_stream(gq + (size_t)c * 16);
-            r.w[b][1] = ldg_stream(uq + (size_t)c * 16);
-            r.sc[b][0] = ldg_f32(gs + (c >> 1));
-            r.sc[b][1] = ldg_f32(us + (c >> 1));
-        }
+        r.w[b][0] = ldg_stream(gq + (b0 + b) * 512);
+        r.w[b][1] = ldg_stream(uq + (b0 + b) * 512);
+        r.sc[b][0] = ldg_f32(gs + (b0 + b) * 16);
+        r.sc[b][1] = ldg_f32(us + (b0 + b) * 16);
     }
 }
 
-__device__ __forceinline__ void half_compute(const StageGeom& g, const float4* xs, const float* corr, int b0,
-                                             int lane, const HalfRegs& r, float& tg, float& tu)
+template <int b0>
+__device__ __forceinline__ void half_compute(const float4* xs, const float* corr, const int (&off)[8],
+                                             const HalfRegs& r, float& tg, float& tu)
 {
+    // xs: staged x; corr: this lane's chunk corrections (corr + lane)
 #pragma unroll
     for (int b = 0; b < kHalf; ++b) {
-        const int c = lane + 32 * (b0 + b);
-        if (b0 + b < g.per_lane && c < g.nch) {
-            float2 acc[2];
-            chunk_acc_rows<2>(r.w[b], xs + (b0 + b) * 256, lane, acc);
-            const float cr = corr[c];
-            tg = chunk_finish(acc[0], cr, r.sc[b][0], tg);
-            tu = chunk_finish(acc[1], cr, r.sc[b][1], tu);
-        }
+        float2 acc[2];
+        chunk_acc_rows_off<2>(r.w[b], xs + (b0 + b) * 256, off, acc);
+        const float cr = corr[(b0 + b) * 32];
+        tg = chunk_finish(acc[0], cr, r.sc[b][0], tg);
+        tu = chunk_finish(acc[1], cr, r.sc[b][1], tu);
     }
 }
 
-// One work unit = (slot, row n): gu[slot][0][n] = (W_gate,e x)[n] and
-// gu[slot][1][n] = (W_up,e x)[n]; SwiGLU is applied when the down kernel stages
-// h.  The gate and up rows share every staged x load.  Units are numbered
-// shared expert first, then routed slots, rows fastest, and dealt out
-// statically (warp gw of W takes gw, gw + W, ...): all units cost the same.
-// The multiply-adds of the int4 decode keep the integer pipe busy, so the kernel
-// relies on occupancy (32 warps per SM at <= 64 registers) to keep enough
-// loads in flight; each half-row's loads are issued together.  A warp whose
-// first unit is a shared-expert row issues its loads before the router's top-k
-// is known; warp 0's top-k and the staging of x overlap them.
+// One work unit = (slot, row n): h[slot][n] = silu((W_gate,e x)[n]) * (W_up,e x)[n];
+// the gate and up rows share every staged x load.  Units are numbered shared
+// expert first, then routed slots, rows fastest, and dealt out statically (warp
+// gw of W takes gw, gw + W, ...): all units cost the same.  The int4 decode
+// keeps the integer pipe busy, so the kernel relies on occupancy (32 warps per
+// SM at <= 64 registers) to keep loads in flight; each half-row's loads are
+// issued together.  A warp whose first unit is a shared-expert row issues its
+// loads before the router's top-k is known; the staging of x and warp 0's
+// top-k overlap them.  kPL = chunks per lane = H / 1024 (two halves of kHalf).
 template <bool kBf16>
 __global__ void __launch_bounds__(kSingleThreads, 2)
 gateup_single_kernel(SingleArgs a)
 {
+    constexpr int kPL = 2 * kHalf;
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_e[kMaxTopK + 1];
     __shared__ int32_t s_idx[kMaxTopK];
     __shared__ float s_w[kMaxTopK];
-    const StageGeom g = stage_geom(a.H);
+    const StageGeom g = stage_geom(a.H);  // g.per_lane == kPL on this path
     float4* xs = reinterpret_cast<float4*>(smem);
     float* corr = reinterpret_cast<float*>(smem + (size_t)g.f4 * 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = gridDim.x * kSingleWarps;
+    int off[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) off[j] = j * 32 + (lane ^ j);
+    const size_t qrow = (size_t)a.H / 2, srow = (size_t)a.H / kGroup;
+    auto rows = [&](int e, int n, const uint8_t*& gq, const uint8_t*& uq, const float*& gs, const float*& us) {
+        const size_t row = (size_t)e * a.F + n;
+        gq = a.gate_q + row * qrow + lane * 16;
+        uq = a.up_q + row * qrow + lane * 16;
+        gs = a.gate_s + row * srow + (lane >> 1);
+        us = a.up_s + row * srow + (lane >> 1);
+    };
 
     int u = blockIdx.x * kSingleWarps + warp;
     HalfRegs A;
     const bool first_shared = u < a.F;
-    if (first_shared) half_load(a, g, a.E, u, 0, lane, A);  // shared expert: no routing needed
+    if (first_shared) {  // shared expert: no routing needed
+        const uint8_t *gq, *uq;
+        const float *gs, *us;
+        rows(a.E, u, gq, uq, gs, us);
+        half_load<0>(gq, uq, gs, us, A);
+    }
     stage_vectors<kBf16>(a.x, a.H, 1, [](int) { return 0; }, g, xs, corr);  // x is this call's input
     griddep_wait();  // router scores of this call are complete
     if (warp == 0) {
@@ -131,16 +140,17 @@ gateup_single_kernel(SingleArgs a)
 
     bool loaded = first_shared;
     int sl = u / a.F, n = u - sl * a.F;  // slot index (0 = shared) and row of unit u
+    const float* cl = corr + lane;
     while (sl <= a.k) {
-        const int e = sl == 0 ? a.E : s_e[sl - 1];
+        const uint8_t *gq, *uq;
+        const float *gs, *us;
+        rows(sl == 0 ? a.E : s_e[sl - 1], n, gq, uq, gs, us);
         float tg = 0.f, tu = 0.f;
-        if (!loaded) half_load(a, g, e, n, 0, lane, A);
+        if (!loaded) half_load<0>(gq, uq, gs, us, A);
         loaded = false;
-        half_compute(g, xs, corr, 0, lane, A, tg, tu);
-        if (g.per_lane > kHalf) {
-            half_load(a, g, e, n, kHalf, lane, A);
-            half_compute(g, xs, corr, kHalf, lane, A, tg, tu);
-        }
+        half_compute<0>(xs, cl, off, A, tg, tu);
+        half_load<kHalf>(gq, uq, gs, us, A);
+        half_compute<kHalf>(xs, cl, off, A, tg, tu);
         tg = warp_sum(tg);
         tu = warp_sum(tu);
         if (lane == 0) {
@@ -157,43 +167,39 @@ gateup_single_kernel(SingleArgs a)
 }
 
 // Loads of one down item: rows n, n+1 of expert e's down matrix, the lane's
-// chunks c = lane + 32 i (i < per_lane <= 2).
+// chunks c = lane + 32 i (i < 2: F = 2048 on this path).
 struct DownRegs {
     uint4 w[2][2];  // [row][i]
     float sc[2][2];
 };
 
-__device__ __forceinline__ void down_load(const SingleArgs& a, const StageGeom& g, int e, int n, int lane,
-                                          DownRegs& r)
+__device__ __forceinline__ void down_load(const SingleArgs& a, int e, int n, int lane, DownRegs& r)
 {
+    const size_t row = (size_t)e * a.H + n;
+    const uint8_t* q = a.down_q + row * ((size_t)a.F / 2) + lane * 16;
+    const float* s = a.down_s + row * ((size_t)a.F / kGroup) + (lane >> 1);
+    const size_t qr = (size_t)a.F / 2, sr = (size_t)a.F / kGroup;
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        const size_t row = (size_t)e * a.H + n + rr;
+    for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-            const int c = lane + 32 * i;
-            if (i < g.per_lane && c < g.nch) {
-                r.w[rr][i] = ldg_stream(a.down_q + row * ((size_t)a.F / 2) + (size_t)c * 16);
-                r.sc[rr][i] = ldg_f32(a.down_s + row * ((size_t)a.F / kGroup) + (c >> 1));
-            }
+            r.w[rr][i] = ldg_stream(q + rr * qr + i * 512);
+            r.sc[rr][i] = ldg_f32(s + rr * sr + i * 16);
         }
-    }
 }
 
-__device__ __forceinline__ void down_compute(const StageGeom& g, const float4* hs, const float* corr, int j,
-                                             float wj, int lane, const DownRegs& r, float& o0, float& o1)
+__device__ __forceinline__ void down_compute(const float4* hs_j, const float* corr_j, const int (&off)[8], float wj,
+                                             const DownRegs& r, float& o0, float& o1)
 {
+    // hs_j: staged h of slot j; corr_j: its chunk corrections + lane
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const int c = lane + 32 * i;
-        if (i < g.per_lane && c < g.nch) {
-            float2 acc[2];
-            const uint4 w2[2] = {r.w[0][i], r.w[1][i]};
-            chunk_acc_rows<2>(w2, hs + (size_t)j * g.f4 + i * 256, lane, acc);
-            const float cr = corr[j * g.nch + c];
-            o0 = fmaf(wj, chunk_finish(acc[0], cr, r.sc[0][i], 0.f), o0);
-            o1 = fmaf(wj, chunk_finish(acc[1], cr, r.sc[1][i], 0.f), o1);
-        }
+        float2 acc[2];
+        const uint4 w2[2] = {r.w[0][i], r.w[1][i]};
+        chunk_acc_rows_off<2>(w2, hs_j + i * 256, off, acc);
+        const float cr = corr_j[i * 32];
+        o0 = fmaf(wj, chunk_finish(acc[0], cr, r.sc[0][i], 0.f), o0);
+        o1 = fmaf(wj, chunk_finish(acc[1], cr, r.sc[1][i], 0.f), o1);
     }
 }
 
@@ -211,12 +217,15 @@ down_single_kernel(SingleArgs a)
     __shared__ int s_e[kMaxTopK + 1];
     __shared__ float s_w[kMaxTopK + 1];
     const int S = a.k + 1;  // slots: k routed + shared
-    const StageGeom g = stage_geom(a.F);
+    const StageGeom g = stage_geom(a.F);  // g.per_lane == 2 on this path
     float4* hs = reinterpret_cast<float4*>(smem);
     float* corr = reinterpret_cast<float*>(smem + (size_t)S * g.f4 * 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = gridDim.x * kSingleWarps;
     const int units = (a.H / 2) * S;
+    int off[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) off[jj] = jj * 32 + (lane ^ jj);
 
     griddep_wait();  // routing and h of this call are complete
     if (threadIdx.x < S) {
@@ -227,14 +236,14 @@ down_single_kernel(SingleArgs a)
     int u = blockIdx.x * kSingleWarps + warp;
     int j = u % S, rp = u / S;  // slot and row pair of unit u
     DownRegs X;
-    if (u < units) down_load(a, g, s_e[j], 2 * rp, lane, X);
+    if (u < units) down_load(a, s_e[j], 2 * rp, lane, X);
     stage_vectors<false>(a.h, a.F, S, [](int t) { return t; }, g, hs, corr);
     __syncthreads();
 
     const int dj = W % S, drp = W / S;  // unit stride W as (slot, row pair) steps
     for (; u < units; u += W) {
         float o0 = 0.f, o1 = 0.f;
-        down_compute(g, hs, corr, j, s_w[j], lane, X, o0, o1);
+        down_compute(hs + (size_t)j * g.f4, corr + j * g.nch + lane, off, s_w[j], X, o0, o1);
         const int jc = j, nc = 2 * rp;
         j += dj;
         rp += drp;
@@ -242,7 +251,7 @@ down_single_kernel(SingleArgs a)
             j -= S;
             ++rp;
         }
-        if (u + W < units) down_load(a, g, s_e[j], 2 * rp, lane, X);
+        if (u + W < units) down_load(a, s_e[j], 2 * rp, lane, X);
         o0 = warp_sum(o0);
         o1 = warp_sum(o1);
         if (lane == 0) {

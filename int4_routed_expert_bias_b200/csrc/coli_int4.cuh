@@ -77,6 +77,26 @@ __device__ __forceinline__ void chunk_acc_rows(const uint4 (&w)[NS], const float
     }
 }
 
+// Same, with the lane's 8 swizzled slot offsets (slot j of row block 0 at
+// xrow[off[j]], off[j] = j * 32 + (lane ^ j)) computed once by the caller.
+template <int NS>
+__device__ __forceinline__ void chunk_acc_rows_off(const uint4 (&w)[NS], const float4* xrow, const int (&off)[8],
+                                                   float2 (&acc)[NS])
+{
+#pragma unroll
+    for (int r = 0; r < NS; ++r) acc[r] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 xlo = xrow[off[2 * q]];
+        const float4 xhi = xrow[off[2 * q + 1]];
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {
+            const uint32_t wd = q == 0 ? w[r].x : q == 1 ? w[r].y : q == 2 ? w[r].z : w[r].w;
+            acc[r] = word_dot(wd, xlo, xhi, acc[r]);
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Staging of activation vectors in shared memory.
 //
