@@ -15,6 +15,7 @@
 #include "coli_common.cuh"
 #include "coli_decode.cuh"
 #include "coli_decode1.cuh"
+#include "coli_prefill.cuh"
 #include "coli_router.cuh"
 #include "coli_union.cuh"
 
@@ -95,7 +96,10 @@ coli_status device_info(DeviceInfo** out)
             (e = allow_smem(expert_phase_kernel<false, false, 4>, lim)) != cudaSuccess ||
             (e = allow_smem(gateup_single_kernel<false>, lim)) != cudaSuccess ||
             (e = allow_smem(gateup_single_kernel<true>, lim)) != cudaSuccess ||
-            (e = allow_smem(down_single_kernel<0>, lim)) != cudaSuccess)
+            (e = allow_smem(down_single_kernel<0>, lim)) != cudaSuccess ||
+            (e = allow_smem(prefill_gemm_kernel<true, true>, (int)kPfSmemBytes)) != cudaSuccess ||
+            (e = allow_smem(prefill_gemm_kernel<true, false>, (int)kPfSmemBytes)) != cudaSuccess ||
+            (e = allow_smem(prefill_gemm_kernel<false, true>, (int)kPfSmemBytes)) != cudaSuccess)
             return cuda_fail(e, "kernel attribute setup");
         d.smem_optin = lim;
         d.ready = true;
@@ -238,6 +242,9 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem,
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
+
+// Batches above this size take the tensor-core prefill path.
+constexpr int kDecodeMaxT = 64;
 
 // Batches up to this size take the top-k inside the union block.
 constexpr int kFusedTopkMaxT = 256;
@@ -385,6 +392,55 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
             e = ot == COLI_BF16 ? launch_pdl(combine_single_kernel<true>, blocks, 128, 0, stream, w.partial, k + 1, H, out)
                                 : launch_pdl(combine_single_kernel<false>, blocks, 128, 0, stream, w.partial, k + 1, H, out);
             if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+        }
+        if ((e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
+        e = cudaGetLastError();
+        return e == cudaSuccess ? COLI_OK : cuda_fail(e, "layer launch");
+    }
+
+    if (T > kDecodeMaxT && H % 128 == 0 && (size_t)dev->smem_optin >= kPfSmemBytes) {
+        // Prefill: tensor-core grouped GEMMs over token tiles of <= 256 pairs per expert
+        if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
+        {
+            dim3 grid((T + kRtTile - 1) / kRtTile, (E + kRtTile - 1) / kRtTile);
+            if (bf16) router_logits_tiled_kernel<true><<<grid, 256, 0, stream>>>(x, T, H, L->w_router, E, w.logits);
+            else router_logits_tiled_kernel<false><<<grid, 256, 0, stream>>>(x, T, H, L->w_router, E, w.logits);
+        }
+        const bool fused = T <= kFusedTopkMaxT && E <= 256;
+        if (!fused)
+            router_topk_kernel<<<(T + 7) / 8, 256, 0, stream>>>(w.logits, T, E, k, L->sel_bias, L->routed_scale, idx, wt);
+        if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess)
+            return cuda_fail(e, "event record");
+        WorkLists wl{w.pair_token, w.pair_w, w.ctl, w.g_expert, w.g_start, w.g_count, wt, kPfMaxN};
+        TopkArgs tk{w.logits, L->sel_bias, L->routed_scale, wt};
+        if (fused)
+            union_kernel<true, true><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
+                                                                      w.n_active, w.perm, w.inv_perm, wl, tk);
+        else
+            union_kernel<true, false><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
+                                                                       w.n_active, w.perm, w.inv_perm, wl, tk);
+        if ((e = tm.rec(COLI_STAGE_UNION, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_GATEUP, 0)) != cudaSuccess)
+            return cuda_fail(e, "event record");
+        const int P = T * k;
+        const int max_tiles = P / kPfMaxN + E + (T + kPfMaxN - 1) / kPfMaxN + 1;  // >= number of union groups
+        uint16_t* hb = reinterpret_cast<uint16_t*>(w.h);
+        uint16_t* ys = reinterpret_cast<uint16_t*>(w.partial);
+        PrefillArgs pa{L->gate_q, L->gate_s, L->up_q, L->up_s, F, H, E, k, T, P, x, w.ctl, w.g_expert, w.g_start,
+                       w.g_count, w.pair_token, w.pair_w, w.perm, hb, ys, w.ctl + 3};
+        if (bf16) prefill_gemm_kernel<true, true><<<max_tiles * (2 * F / 128), kPfThreads, kPfSmemBytes, stream>>>(pa);
+        else prefill_gemm_kernel<true, false><<<max_tiles * (2 * F / 128), kPfThreads, kPfSmemBytes, stream>>>(pa);
+        if ((e = tm.rec(COLI_STAGE_GATEUP, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_DOWN, 0)) != cudaSuccess)
+            return cuda_fail(e, "event record");
+        PrefillArgs pd{L->down_q, L->down_s, nullptr, nullptr, H, F, E, k, T, P, hb, w.ctl, w.g_expert, w.g_start,
+                       w.g_count, w.pair_token, w.pair_w, w.perm, hb, ys, w.ctl + 3};
+        prefill_gemm_kernel<false, true><<<max_tiles * (H / 128), kPfThreads, kPfSmemBytes, stream>>>(pd);
+        if ((e = tm.rec(COLI_STAGE_DOWN, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_COMBINE, 0)) != cudaSuccess)
+            return cuda_fail(e, "event record");
+        {
+            const size_t n8 = (size_t)T * H / 8;
+            const int blocks = (int)((n8 + 255) / 256);
+            if (ot == COLI_BF16) slot_reduce_kernel<true><<<blocks, 256, 0, stream>>>(ys, T, k + 1, H, out);
+            else slot_reduce_kernel<false><<<blocks, 256, 0, stream>>>(ys, T, k + 1, H, out);
         }
         if ((e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
         e = cudaGetLastError();

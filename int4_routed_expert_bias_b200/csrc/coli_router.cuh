@@ -79,6 +79,53 @@ router_logits_kernel(const void* __restrict__ x, int T, int H, const float* __re
     }
 }
 
+// logits[t, e] for large batches: a 64-token x 64-expert tile per block,
+// K-steps of 32 staged in shared memory, 4 x 4 outputs per thread, fp32.
+constexpr int kRtTile = 64;
+constexpr int kRtK = 32;
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256)
+router_logits_tiled_kernel(const void* __restrict__ x, int T, int H, const float* __restrict__ w_router, int E,
+                           float* __restrict__ logits)
+{
+    __shared__ float xs[kRtK][kRtTile + 4];
+    __shared__ float ws[kRtK][kRtTile + 4];
+    const int t0 = blockIdx.x * kRtTile, e0 = blockIdx.y * kRtTile;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // outputs (t0 + ty*4 + i, e0 + tx*4 + j)
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < H; k0 += kRtK) {
+        // stage 64 x 32 of x and of w_router, transposed to [k][row]
+        for (int i = threadIdx.x; i < kRtTile * kRtK / 4; i += 256) {
+            const int r = i / (kRtK / 4), c = (i % (kRtK / 4)) * 4;
+            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t0 + r < T) xv = load_act4<kBf16>(static_cast<const char*>(x) + (size_t)(t0 + r) * H * (kBf16 ? 2 : 4), k0 + c);
+            if (e0 + r < E) wv = *reinterpret_cast<const float4*>(w_router + (size_t)(e0 + r) * H + k0 + c);
+            xs[c][r] = xv.x; xs[c + 1][r] = xv.y; xs[c + 2][r] = xv.z; xs[c + 3][r] = xv.w;
+            ws[c][r] = wv.x; ws[c + 1][r] = wv.y; ws[c + 2][r] = wv.z; ws[c + 3][r] = wv.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kRtK; ++kk) {
+            const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+            const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
+            if (t < T && e < E) logits[(size_t)t * E + e] = acc[i][j];
+        }
+}
+
 // Top-k of one token by one warp: sigmoid, bias, k rounds of warp arg-max,
 // renormalised weights.  Lane j keeps the j-th selection.  The arg-max key is
 // (c desc, index asc); a non-finite score can never make the warp pick an index

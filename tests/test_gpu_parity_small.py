@@ -142,7 +142,8 @@ def test_ragged_batches(env, T):
     ridx, rw, rout = oracle.moe_layer(x, c.H, c.F, c.E, c.k, c.routed_scale, w_router, sel_bias, ex)
     assert np.array_equal(idx, ridx)
     np.testing.assert_allclose(w, rw, rtol=2e-6)
-    assert S.rel_inf_err(out, rout) <= S.TOL_DECODE
+    # batches above 64 tokens take the bf16 tensor-core prefill path
+    assert S.rel_inf_err(out, rout) <= (S.TOL_DECODE if T <= 64 else S.TOL_PREFILL)
 
 
 def test_smallest_shapes_bf16_in_bf16_out(env):
