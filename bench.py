@@ -58,11 +58,13 @@ def parse():
 
 
 def measured_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, kind)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return (d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0),
+                "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 def workload_desc(c):
@@ -228,8 +230,8 @@ def run_reference(args):
 # our arm
 
 def traffic_from_profiles(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (hash match); else None."""
+    """DRAM bytes per launch from the committed ncu summary profiles/<kernel>_<workload>.txt,
+    if the kernel sources it lists still hash to the recorded value; else None."""
     import hashlib
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.txt")
     if not os.path.exists(p):
@@ -239,10 +241,15 @@ def traffic_from_profiles(kernel, workload):
         if ":" in line:
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
+    files = kv.get("source_files", "").split()
+    if not files:
+        return None
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "int4_routed_expert_bias_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in files:
+        fp = os.path.join(ROOT, f)
+        if not os.path.exists(fp):
+            return None
+        h.update(open(fp, "rb").read())
     if kv.get("source_sha256") != h.hexdigest()[:16]:
         return None
     try:
@@ -269,7 +276,7 @@ def run_ours(args):
         c = inputs.Config(c.cfg, f"{c.name}-E{args.experts}", c.H, c.F, args.experts, c.k, c.T, c.x_dtype,
                           c.out_dtype, args.layers)
     seed = SEED + 1000 * rank
-    hbm_peak, _, peak_kind = measured_peaks()
+    hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
 
     # eight resident layers, expert weights generated on the device
     layers, bufs, routers = [], [], []
@@ -365,23 +372,37 @@ def run_ours(args):
     layer_alg = float(np.mean((U + 1) * c.expert_bytes)) + c.E * c.H * 4 + c.E * 4 + x_bytes \
         + c.T * c.H * (2 if c.out_dtype == "bf16" else 4)
     layer_gbs = layer_alg / (ms_per_step * 1e-3) / 1e9
-    traffic = traffic_from_profiles("gateup", c.name)
+    traffic = traffic_from_profiles("gateup", c.name) if c.T <= 64 else traffic_from_profiles("gateup-gemm", c.name)
+
+    prefill = c.T > 64
+    if prefill:
+        # dominant kernel: the gate/up grouped GEMM, 2 * (pairs + shared) * 2F * H flops
+        gu_flops = 2.0 * (c.T * c.k + c.T) * (2 * c.F) * c.H
+        gu_tflops = gu_flops / (stage_ms["gateup"] * 1e-3) / 1e12
+        roofline = {"kernel": "prefill_gemm_kernel<gate/up> (tcgen05 int4-dequant grouped GEMM + SwiGLU)",
+                    "bound": "tensor", "achieved": gu_tflops, "peak": bf16_sust, "unit": "TFLOP/s",
+                    "frac": gu_tflops / bf16_sust, "traffic": traffic, "peak_kind": peak_kind + " (sustained bf16)",
+                    "alg_flops_per_launch": gu_flops}
+    else:
+        roofline = {"kernel": ("gateup_single_kernel" if c.T == 1 else "expert_phase_kernel<gateup>")
+                    + " (gate/up + SwiGLU, routed and shared experts)",
+                    "bound": "hbm", "achieved": gu_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": gu_gbs / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
+                    "alg_bytes_per_launch": gu_alg}
+    extra = {"graph_calls": G, "parallelism": f"replicas x{world}", "mean_union_U": float(U.mean()),
+             "layer_alg_bytes_per_call": layer_alg, "layer_gbs": layer_gbs,
+             "layer_frac_of_hbm_peak": layer_gbs / hbm_peak, "stage_ms": stage_ms}
+    if prefill:
+        layer_flops = 2.0 * (c.T * c.k + c.T) * 3 * c.F * c.H + 2.0 * c.T * c.E * c.H
+        extra["layer_tflops"] = layer_flops / (ms_per_step * 1e-3) / 1e12
+        extra["layer_frac_of_bf16_sustained"] = extra["layer_tflops"] / bf16_sust
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32" if c.T <= 64 else "f32", "data": "synthetic",
-            "config": config_block(c, G, {"graph_calls": G, "parallelism": f"replicas x{world}",
-                                          "mean_union_U": float(U.mean()),
-                                          "layer_alg_bytes_per_call": layer_alg,
-                                          "layer_gbs": layer_gbs,
-                                          "layer_frac_of_hbm_peak": layer_gbs / hbm_peak,
-                                          "stage_ms": stage_ms}),
-            "roofline": {"kernel": ("gateup_single_kernel" if c.T == 1 else "expert_phase_kernel<gateup>")
-                         + " (gate/up + SwiGLU, routed and shared experts)",
-                         "bound": "hbm", "achieved": gu_gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": gu_gbs / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
-                         "alg_bytes_per_launch": gu_alg},
+            "dtype": "bf16" if prefill else "f32", "data": "synthetic",
+            "config": config_block(c, G, extra),
+            "roofline": roofline,
             "gpu_launches": steps * kernels_per_call(c.T, c.E),
             "clocks": clocks}
 

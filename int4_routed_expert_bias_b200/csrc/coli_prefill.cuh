@@ -31,7 +31,8 @@
 
 namespace coli {
 
-constexpr int kPfStages = 4;
+constexpr int kPfStages = 3;    // MMA stages (bf16 weights + token rows)
+constexpr int kPfRawStages = 8; // int4 byte stages (issued kPfRawStages - 1 k-steps ahead)
 constexpr int kPfProducers = 256;            // 8 producer warps
 constexpr int kPfThreads = kPfProducers + 32;  // + the MMA warp
 constexpr int kPfMaxN = 256;                 // tokens per tile
@@ -40,8 +41,9 @@ constexpr int kPfKStep = 64;                 // = one scale group
 constexpr int kPfABytes = 128 * 128;         // 128 rows x 64 bf16
 constexpr int kPfBBytes = kPfMaxN * 128;     // 256 rows x 64 bf16
 constexpr int kPfRawBytes = 128 * 32 + 128 * 2 * 4;  // int4 bytes + two copies of the scale per row
-constexpr int kPfStageBytes = kPfABytes + kPfBBytes + kPfRawBytes;
-constexpr size_t kPfSmemBytes = 1024 /*alignment slack*/ + (size_t)kPfStages * kPfStageBytes + 256;
+constexpr int kPfStageBytes = kPfABytes + kPfBBytes;
+constexpr size_t kPfSmemBytes =
+    1024 /*alignment slack*/ + (size_t)kPfStages * kPfStageBytes + (size_t)kPfRawStages * kPfRawBytes + 256;
 constexpr unsigned long long kPfWaitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 // ---------------------------------------------------------------------------
@@ -103,6 +105,11 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// The mbarrier receives one arrival when all earlier cp.async of this thread land.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
@@ -233,7 +240,7 @@ prefill_gemm_kernel(PrefillArgs a)
 
     auto stage_a = [&](int s) { return smem + (size_t)s * kPfStageBytes; };
     auto stage_b = [&](int s) { return smem + (size_t)s * kPfStageBytes + kPfABytes; };
-    auto stage_raw = [&](int s) { return smem + (size_t)s * kPfStageBytes + kPfABytes + kPfBBytes; };
+    auto stage_raw = [&](int r) { return smem + (size_t)kPfStages * kPfStageBytes + (size_t)r * kPfRawBytes; };
 
     if (warp < 8) {
         // ---------------- producers ----------------
@@ -256,42 +263,54 @@ prefill_gemm_kernel(PrefillArgs a)
         const size_t act_row_bytes = (size_t)a.K * ((kGemm1 && !kXBf16) ? 4 : 2);
         bool ok = true;
 
-        auto issue = [&](int ks) {  // cp.async the raw data of k-step ks into its stage
-            const int s = ks % kPfStages;
-            unsigned char* raw = stage_raw(s);
+        // int4 bytes and scales of k-step ks -> raw ring slot ks % kPfRawStages (own data of this thread)
+        auto issue_raw = [&](int ks) {
+            unsigned char* raw = stage_raw(ks % kPfRawStages);
             cp_async16(raw + row * 32 + half * 16, qrow + (size_t)ks * 32 + half * 16);
             cp_async4(raw + 128 * 32 + (row * 2 + half) * 4, srow + ks);
-            if (kGemm1 && !kXBf16) {
-                // fp32 activations are converted while storing (plain loads)
-            } else {
-                unsigned char* b = stage_b(s);
-                for (int i = tid; i < N * 8; i += kPfProducers) {
-                    const int r = i >> 3, c = i & 7;
-                    const int src_row = s_tok[r] >= 0 ? s_tok[r] : s_tok[0];
-                    const unsigned char* src = static_cast<const unsigned char*>(a.act) +
-                                               (size_t)src_row * act_row_bytes + (size_t)ks * 128 + c * 16;
-                    cp_async16(b + r * 128 + ((c ^ (r & 7)) * 16), src);
-                }
+        };
+        // token rows of k-step ks -> MMA stage ks % kPfStages; the stage's full barrier gets
+        // this thread's arrival when its copies (and all earlier ones) have landed
+        auto issue_b = [&](int ks) {
+            const int s = ks % kPfStages;
+            if (kGemm1 && !kXBf16) return;  // fp32 activations: converted while storing, below
+            unsigned char* b = stage_b(s);
+            for (int i = tid; i < N * 8; i += kPfProducers) {
+                const int r = i >> 3, c = i & 7;
+                const int src_row = s_tok[r] >= 0 ? s_tok[r] : s_tok[0];
+                const unsigned char* src = static_cast<const unsigned char*>(a.act) + (size_t)src_row * act_row_bytes +
+                                           (size_t)ks * 128 + c * 16;
+                cp_async16(b + r * 128 + ((c ^ (r & 7)) * 16), src);
             }
-            cp_async_commit();
         };
 
-        for (int ks = 0; ks < kPfStages - 1 && ks < ksteps; ++ks) issue(ks);
+        // prologue: int4 bytes kPfRawStages - 1 k-steps ahead, token rows kPfStages - 1 ahead
+        for (int ks = 0; ks < kPfRawStages - 1; ++ks) {
+            if (ks < ksteps) issue_raw(ks);
+            cp_async_commit();
+        }
+        for (int ks = 0; ks < kPfStages - 1 && ks < ksteps; ++ks) {
+            issue_b(ks);
+            if (kGemm1 && !kXBf16) mbar_arrive(&full_bar[ks % kPfStages]);
+            else cp_async_arrive_noinc(&full_bar[ks % kPfStages]);
+        }
         for (int ks = 0; ks < ksteps && ok; ++ks) {
             const int s = ks % kPfStages;
-            // refill the stage that k-step ks + S - 1 uses once the MMA has released it
-            const int kn = ks + kPfStages - 1;
-            if (kn < ksteps) {
-                const int sn = kn % kPfStages, fill = kn / kPfStages;
-                if (fill > 0) ok = mbar_wait(&empty_bar[sn], (fill - 1) & 1, deadline, a.err);
+            // token rows for k-step ks + S - 1, once the MMA has released that stage
+            const int kb = ks + kPfStages - 1;
+            if (kb < ksteps) {
+                const int sb = kb % kPfStages, fill = kb / kPfStages;
+                if (fill > 0) ok = mbar_wait(&empty_bar[sb], (fill - 1) & 1, deadline, a.err);
                 if (!ok) break;
-                issue(kn);
-                cp_async_wait<kPfStages - 1>();
-            } else {
-                cp_async_wait<0>();
+                issue_b(kb);
+                if (kGemm1 && !kXBf16) mbar_arrive(&full_bar[sb]);
+                else cp_async_arrive_noinc(&full_bar[sb]);
             }
-            // k-step ks: its raw bytes (and token rows) have landed
-            unsigned char* raw = stage_raw(s);
+            // int4 bytes for k-step ks + R - 1 (its ring slot was consumed at k-step ks - 1)
+            if (ks + kPfRawStages - 1 < ksteps) issue_raw(ks + kPfRawStages - 1);
+            cp_async_commit();
+            cp_async_wait<kPfRawStages - 1>();  // the group of k-step ks has landed
+            unsigned char* raw = stage_raw(ks % kPfRawStages);
             const uint4 w = *reinterpret_cast<const uint4*>(raw + row * 32 + half * 16);
             const float sc = *reinterpret_cast<const float*>(raw + 128 * 32 + (row * 2 + half) * 4);
             unsigned char* A = stage_a(s);
@@ -327,7 +346,6 @@ prefill_gemm_kernel(PrefillArgs a)
                 }
             }
             fence_proxy_async();
-            mbar_arrive(&full_bar[s]);
             mbar_arrive(&full_bar[s]);
         }
         cp_async_wait<0>();
