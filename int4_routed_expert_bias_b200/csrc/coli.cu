@@ -4,7 +4,9 @@
 // kernel selection and launch order.  Every step of the layer runs in the
 // kernels of this library; there is no CPU fallback.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -97,9 +99,9 @@ coli_status device_info(DeviceInfo** out)
             (e = allow_smem(gateup_single_kernel<false>, lim)) != cudaSuccess ||
             (e = allow_smem(gateup_single_kernel<true>, lim)) != cudaSuccess ||
             (e = allow_smem(down_single_kernel<0>, lim)) != cudaSuccess ||
-            (e = allow_smem(prefill_gemm_kernel<true, true>, (int)kPfSmemBytes)) != cudaSuccess ||
-            (e = allow_smem(prefill_gemm_kernel<true, false>, (int)kPfSmemBytes)) != cudaSuccess ||
-            (e = allow_smem(prefill_gemm_kernel<false, true>, (int)kPfSmemBytes)) != cudaSuccess)
+            (kPfSmemBytes <= (size_t)lim &&
+             ((e = allow_smem(prefill_gemm_kernel<true>, (int)kPfSmemBytes)) != cudaSuccess ||
+              (e = allow_smem(prefill_gemm_kernel<false>, (int)kPfSmemBytes)) != cudaSuccess)))
             return cuda_fail(e, "kernel attribute setup");
         d.smem_optin = lim;
         d.ready = true;
@@ -241,6 +243,47 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once (the library links
+// only the runtime).  nullptr when the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Row-major 2-D tensor [rows, inner] of esize-byte elements, read in boxes of
+// box_inner x box_rows.
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base, uint64_t inner,
+               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * esize};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Maps of one expert matrix set: int4 bytes [(E+1) NW, K/2] and scales [(E+1) NW, K/64].
+bool encode_weight_maps(CUtensorMap* q, CUtensorMap* s, const uint8_t* qp, const float* sp, int E, int NW, int K)
+{
+    const uint64_t rows = (uint64_t)(E + 1) * NW;
+    return encode_2d(q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qp, (uint64_t)K / 2, rows, kPfRawK / 2, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+           encode_2d(s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sp, (uint64_t)K / kGroup, rows, kPfRawK / kGroup, 64,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // Batches above this size take the tensor-core prefill path.
@@ -398,8 +441,22 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
         return e == cudaSuccess ? COLI_OK : cuda_fail(e, "layer launch");
     }
 
-    if (T > kDecodeMaxT && H % 128 == 0 && (size_t)dev->smem_optin >= kPfSmemBytes) {
-        // Prefill: tensor-core grouped GEMMs over token tiles of <= 256 pairs per expert
+    // Prefill: tensor-core grouped GEMMs over token tiles of <= kPfMaxN pairs per expert.
+    // The TMA maps need K a multiple of 256 (scale rows of whole 16-byte boxes).
+    CUtensorMap m_gq, m_gs, m_uq, m_us, m_dq, m_ds, m_x, m_h;
+    const size_t Q = (size_t)T * k + T;
+    uint16_t* xg = reinterpret_cast<uint16_t*>(w.partial);  // gathered rows; later reused for ys
+    uint16_t* hb = reinterpret_cast<uint16_t*>(w.h);
+    const bool prefill = T > kDecodeMaxT && H % kPfRawK == 0 && F % kPfRawK == 0 &&
+                         (size_t)dev->smem_optin >= kPfSmemBytes &&
+                         encode_weight_maps(&m_gq, &m_gs, L->gate_q, L->gate_s, E, F, H) &&
+                         encode_weight_maps(&m_uq, &m_us, L->up_q, L->up_s, E, F, H) &&
+                         encode_weight_maps(&m_dq, &m_ds, L->down_q, L->down_s, E, H, F) &&
+                         encode_2d(&m_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xg, (uint64_t)H, Q, kPfKStep, kPfBRows,
+                                   CU_TENSOR_MAP_SWIZZLE_128B) &&
+                         encode_2d(&m_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hb, (uint64_t)F, Q, kPfKStep, kPfBRows,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (prefill) {
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
         {
             dim3 grid((T + kRtTile - 1) / kRtTile, (E + kRtTile - 1) / kRtTile);
@@ -423,17 +480,21 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
             return cuda_fail(e, "event record");
         const int P = T * k;
         const int max_tiles = P / kPfMaxN + E + (T + kPfMaxN - 1) / kPfMaxN + 1;  // >= number of union groups
-        uint16_t* hb = reinterpret_cast<uint16_t*>(w.h);
-        uint16_t* ys = reinterpret_cast<uint16_t*>(w.partial);
-        PrefillArgs pa{L->gate_q, L->gate_s, L->up_q, L->up_s, F, H, E, k, T, P, x, w.ctl, w.g_expert, w.g_start,
-                       w.g_count, w.pair_token, w.pair_w, w.perm, hb, ys, w.ctl + 3};
-        if (bf16) prefill_gemm_kernel<true, true><<<max_tiles * (2 * F / 128), kPfThreads, kPfSmemBytes, stream>>>(pa);
-        else prefill_gemm_kernel<true, false><<<max_tiles * (2 * F / 128), kPfThreads, kPfSmemBytes, stream>>>(pa);
+        {
+            const size_t n = Q * (size_t)(H / 8);
+            const int blocks = (int)((n + 255) / 256);
+            if (bf16) prefill_gather_kernel<true><<<blocks, 256, 0, stream>>>(x, w.pair_token, (int)Q, H, xg);
+            else prefill_gather_kernel<false><<<blocks, 256, 0, stream>>>(x, w.pair_token, (int)Q, H, xg);
+        }
+        PrefillArgs pa{F, H, k, P, F / 64, w.ctl, w.g_expert, w.g_start, w.g_count, w.perm, w.pair_w, hb, xg, w.ctl + 3};
+        const int grid1 = std::min(dev->sms, max_tiles * (F / 64));
+        prefill_gemm_kernel<true><<<grid1, kPfThreads, kPfSmemBytes, stream>>>(m_gq, m_uq, m_gs, m_us, m_x, pa);
         if ((e = tm.rec(COLI_STAGE_GATEUP, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_DOWN, 0)) != cudaSuccess)
             return cuda_fail(e, "event record");
-        PrefillArgs pd{L->down_q, L->down_s, nullptr, nullptr, H, F, E, k, T, P, hb, w.ctl, w.g_expert, w.g_start,
-                       w.g_count, w.pair_token, w.pair_w, w.perm, hb, ys, w.ctl + 3};
-        prefill_gemm_kernel<false, true><<<max_tiles * (H / 128), kPfThreads, kPfSmemBytes, stream>>>(pd);
+        uint16_t* ys = xg;  // the gathered rows are dead once gate/up is done
+        PrefillArgs pd{H, F, k, P, H / 128, w.ctl, w.g_expert, w.g_start, w.g_count, w.perm, w.pair_w, hb, ys, w.ctl + 3};
+        const int grid2 = std::min(dev->sms, max_tiles * (H / 128));
+        prefill_gemm_kernel<false><<<grid2, kPfThreads, kPfSmemBytes, stream>>>(m_dq, m_dq, m_ds, m_ds, m_h, pd);
         if ((e = tm.rec(COLI_STAGE_DOWN, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_COMBINE, 0)) != cudaSuccess)
             return cuda_fail(e, "event record");
         {

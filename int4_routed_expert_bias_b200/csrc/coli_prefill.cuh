@@ -1,5 +1,5 @@
 // coli_prefill.cuh -- expert phases for prefill batches: int4-dequant grouped GEMM
-// on the 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM).
+// on the 5th-generation tensor cores (tcgen05.mma, operands and accumulators in TMEM).
 //
 // The pages compute batched prefill with an int4 kernel and single-token
 // decode in f32 ("Colibri 完全ガイド", section 詳細解説 step 3); with hundreds of
@@ -7,44 +7,63 @@
 // tensor cores here.  Weights are int4 with one fp32 scale per 64 along K
 // ("gs64 build", "colibri: 744B MoEをストレージから推論するCエンジン").
 //
-// One CTA computes one tile D[128 weight rows, N tokens] = W[128, K] . X[N, K]^T
-// for one token tile of one expert (a union group of <= 256 tokens, N padded
-// to a multiple of 16):
-//   - 8 producer warps stage, per K-step of 64, the int4 bytes and scales of the
-//     128 weight rows and the N token rows (bf16) with cp.async, S stages ahead;
-//     the token rows land directly in the 128-byte-swizzled K-major layout the
-//     MMA reads; the int4 bytes are dequantised to bf16 (q * scale) into the
-//     same layout;
-//   - one thread of a 9th warp issues tcgen05.mma (M 128, N, K 16, bf16 in,
-//     fp32 accumulate in TMEM) and tcgen05.commit frees each stage;
-//   - after the last K-step the first four warps read the accumulator with
-//     tcgen05.ld and write the tile: the gate/up GEMM applies SwiGLU (gate and
-//     up rows are interleaved in 32-row blocks of the weight tile); the down
-//     GEMM multiplies by the routing weight and writes one bf16 row per (token,
-//     slot), summed later in slot order (deterministic combine).
-// Every wait on an mbarrier is bounded in time; a timeout sets an error word
-// and the CTA winds down (frees its TMEM) instead of hanging.
+// Work item = one weight tile (128 rows) x one token tile (a union group of
+// <= kPfMaxN pairs of one expert, N padded to 16):  D[128, N] = W[128, K] . X[N, K]^T.
+// Persistent CTAs (one per SM) walk the items; inside a CTA, warp roles:
+//   warp 0     TMA producer: int4 bytes + scales of the weight tile, 256 K at a
+//              time (3-deep ring), and the token rows (bf16), 64 K at a time
+//              (5-deep ring), straight into the 128-byte-swizzled layouts;
+//   warps 6-13 dequantise: each thread owns one weight row (= TMEM lane) and
+//              half of a 64-K step; q * s is formed in bf16 and written into a
+//              4-deep ring of A operands in TMEM with tcgen05.st;
+//   warp 1     one thread issues tcgen05.mma (A from TMEM, B from shared memory,
+//              M 128, K 16, fp32 accumulate) into one of two TMEM accumulators;
+//   warps 2-5  epilogue: tcgen05.ld of the finished accumulator while the next
+//              item accumulates into the other one.  The gate/up GEMM applies
+//              SwiGLU (tile rows 0-63 are gate rows, 64-127 the matching up
+//              rows); the down GEMM scales by the routing weight and writes one
+//              bf16 row per (token, slot), summed later in slot order.
+//
+// K order inside the MMA.  A dequantised register holds the nibbles m and m + 4
+// of a 32-bit word of int4 (bits 4m and 4m + 16), so MMA K position p of each
+// group of 8 carries k = sigma(p), sigma = (0, 4, 1, 5, 2, 6, 3, 7).  The token
+// rows (gathered activations, and the SwiGLU output h that the down GEMM reads)
+// are stored in the same permuted order, so every dot product is unchanged.
+//
+// Every wait on an mbarrier is bounded in time; a timeout sets an error word and
+// every role winds down (in-flight copies land, TMEM is freed) instead of hanging.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (type only; maps are encoded on the host)
+
 #include "coli_common.cuh"
-#include "coli_int4.cuh"
 
 namespace coli {
 
-constexpr int kPfStages = 3;    // MMA stages (bf16 weights + token rows)
-constexpr int kPfRawStages = 8; // int4 byte stages (issued kPfRawStages - 1 k-steps ahead)
-constexpr int kPfProducers = 256;            // 8 producer warps
-constexpr int kPfThreads = kPfProducers + 32;  // + the MMA warp
-constexpr int kPfMaxN = 256;                 // tokens per tile
-constexpr int kPfTmemCols = 256;
-constexpr int kPfKStep = 64;                 // = one scale group
-constexpr int kPfABytes = 128 * 128;         // 128 rows x 64 bf16
-constexpr int kPfBBytes = kPfMaxN * 128;     // 256 rows x 64 bf16
-constexpr int kPfRawBytes = 128 * 32 + 128 * 2 * 4;  // int4 bytes + two copies of the scale per row
-constexpr int kPfStageBytes = kPfABytes + kPfBBytes;
-constexpr size_t kPfSmemBytes =
-    1024 /*alignment slack*/ + (size_t)kPfStages * kPfStageBytes + (size_t)kPfRawStages * kPfRawBytes + 256;
+constexpr int kPfMaxN = 192;      // tokens per tile (union group size on this path)
+constexpr int kPfKStep = 64;      // K per MMA stage = one scale group
+constexpr int kPfRawK = 256;      // K per int4 stage
+constexpr int kPfRawStages = 3;
+constexpr int kPfBStages = 5;
+constexpr int kPfAStages = 4;     // dequantised weight stages in TMEM, 32 columns each
+constexpr int kPfTmemCols = 512;
+constexpr int kPfACol = 2 * kPfMaxN;  // columns [0, 2 N_max): two accumulators; then the A ring
+constexpr int kPfBRows = 32;          // token rows per TMA box
+constexpr int kPfBStageBytes = kPfMaxN * 128;
+constexpr int kPfRawHalfBytes = 64 * kPfRawK / 2;             // int4 bytes of 64 rows
+constexpr int kPfRawScaleOff = 2 * kPfRawHalfBytes;          // then 2 x 64 rows x 4 scales
+constexpr int kPfRawStageBytes = kPfRawScaleOff + 2 * 64 * 16;
+constexpr int kPfXchFloats = 64 * 17;                        // gate/up exchange, one buffer
+constexpr int kPfThreads = 14 * 32;
+constexpr int kPfWarpMma = 1, kPfWarpEpi = 2, kPfWarpDeq = 6;
+constexpr size_t kPfSmemBytes = 1024 /*alignment slack*/ + (size_t)kPfBStages * kPfBStageBytes +
+                                (size_t)kPfRawStages * kPfRawStageBytes + 2 * kPfXchFloats * 4 + 2 * kPfMaxN * 4;
 constexpr unsigned long long kPfWaitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+constexpr unsigned long long kPfDrainNs = 100000000ull;  // teardown waits
+
+static_assert(kPfACol + kPfAStages * 32 <= kPfTmemCols, "TMEM budget");
+static_assert(kPfMaxN % kPfBRows == 0 && kPfMaxN % 16 == 0 && kPfMaxN <= 256, "tile width");
+static_assert(kPfBStageBytes % 1024 == 0 && kPfRawStageBytes % 1024 == 0, "swizzled stages stay 1024-aligned");
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -68,6 +87,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrive once and add `bytes` to the transaction count of the current phase.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok;
@@ -81,7 +107,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the given phase parity; false after the deadline (error word set).
+// Wait for the phase with the given parity to complete; false after the
+// deadline (error word set).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long deadline, int* err)
 {
     if (mbar_try_wait(bar, parity)) return true;
@@ -94,24 +121,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
     return true;
 }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// 2-D tiled TMA load into this CTA's shared memory; completion is counted in
+// bytes on the mbarrier.  x is the innermost coordinate (elements).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src)
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-__device__ __forceinline__ void cp_async4(void* dst, const void* src)
+
+// Named barrier 1 over the 4 epilogue warps; returns the AND of `pred` over them.
+__device__ __forceinline__ bool epi_bar_and(bool pred)
 {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// The mbarrier receives one arrival when all earlier cp.async of this thread land.
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("barrier.cta.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols)
 {
@@ -126,13 +166,15 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+// D[tmem] (+)= A[tmem] . B[smem descriptor]^T
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t acc)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
 __device__ __forceinline__ void tc_commit(uint64_t* bar)
@@ -155,13 +197,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Store 16 consecutive 32-bit TMEM columns of this thread's lane and wait for them.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 bytes,
 // 8-row groups 1024 bytes apart (tcgen05 descriptor version 1).
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFF);  // start address
-    d |= (uint64_t)1 << 16;                  // leading byte offset (16 B units)
+    d |= (uint64_t)1 << 16;                  // leading byte offset (16 B units; unused when swizzled)
     d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset
     d |= (uint64_t)1 << 46;                  // version
     d |= (uint64_t)2 << 61;                  // SWIZZLE_128B
@@ -174,270 +228,335 @@ __device__ __forceinline__ uint32_t idesc_bf16(int n)
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// bf16 bit pattern of q * s for 32 nibbles (16 bytes) of one row.
-__device__ __forceinline__ uint32_t bf16x2_of(float lo, float hi)
+__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
+
+// 32 int4 weights (16 bytes, low nibble first) of one row -> 16 bf16x2 words of
+// q * s.  Word 4i + m holds (nibble m, nibble m + 4) of 32-bit word i: the mask
+// picks bits 0-3 and 16-19 after a shift by 4m, and the xor makes each half the
+// bf16 number 128 + (nibble ^ 8) = 136 + q (exponent 2^7: one unit per step).
+// q = v - 136 is exact; q * bf16(s) is rounded once to bf16.
+__device__ __forceinline__ void dequant32(uint4 w, float s, uint32_t (&o)[16])
 {
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
+    const __nv_bfloat162 s2 = __float2bfloat162_rn(s);
+    const __nv_bfloat162 c136 = __float2bfloat162_rn(136.f);
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            uint32_t v;
+            asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(v) : "r"(words[i] >> (4 * m)), "r"(0x000F000Fu), "r"(0x43084308u));
+            const __nv_bfloat162 q = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&v), c136);
+            o[4 * i + m] = bf16x2_bits(__hmul2(q, s2));
+        }
+    }
+}
+
+// Stored position of feature f in a permuted token row: inverse of sigma inside
+// each group of 8.
+__host__ __device__ __forceinline__ int pf_store_pos(int f)
+{
+    const int m = f & 7;
+    return (f & ~7) | (m < 4 ? 2 * m : 2 * (m - 4) + 1);
 }
 
 struct PrefillArgs {
-    const uint8_t* q0;  // gate (GEMM1) or down (GEMM2) bytes [E+1, N_w, K/2]
-    const float* s0;
-    const uint8_t* q1;  // up bytes (GEMM1)
-    const float* s1;
-    int NW;             // weight rows of one matrix: F (GEMM1: gate and up each) or H (GEMM2)
-    int K;              // H (GEMM1) or F (GEMM2)
-    int E, k, T, P;
-    const void* act;    // GEMM1: x [T, H] (fp32 or bf16); GEMM2: h bf16 [P+T, F]
+    int NW;        // weight rows of one matrix: F (gate/up) or H (down)
+    int K;         // reduction length: H (gate/up) or F (down)
+    int k, P;      // top-k, routed pairs T * k
+    int n_mtiles;  // weight tiles per token tile: F / 64 (gate/up) or H / 128 (down)
     const int32_t* ctl;       // ctl[0] = number of token tiles
-    const int32_t* g_expert;  // token tiles (union groups of <= 256 pairs)
+    const int32_t* g_expert;  // token tiles (union groups of <= kPfMaxN pairs)
     const int32_t* g_start;
     const int32_t* g_count;
-    const int32_t* pair_token;
-    const float* pair_w;
     const int32_t* perm;      // pair id of each sorted position (slot = id % k)
-    uint16_t* h;              // GEMM1 out: h bf16 [P+T, F]
-    uint16_t* ys;             // GEMM2 out: bf16 [T, k+1, H]
+    const float* pair_w;      // routing weight of each sorted position (1 for shared)
+    uint16_t* h;              // gate/up out: bf16 [P + T, F], permuted rows
+    uint16_t* ys;             // down out: bf16 [T, k + 1, H]
     int* err;
 };
 
-template <bool kGemm1, bool kXBf16>
+// tq0 / tq1: int4 bytes of tile rows 0-63 / 64-127 (box 128 B x 64 rows, 128-byte
+// swizzle); ts0 / ts1: their scales (box 4 x 64); tb: token rows, bf16 [P + T, K]
+// permuted (box 64 x 32, 128-byte swizzle).
+template <bool kGemm1>
 __global__ void __launch_bounds__(kPfThreads, 1)
-prefill_gemm_kernel(PrefillArgs a)
+prefill_gemm_kernel(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
+                    const __grid_constant__ CUtensorMap ts0, const __grid_constant__ CUtensorMap ts1,
+                    const __grid_constant__ CUtensorMap tb, const PrefillArgs a)
 {
     extern __shared__ __align__(16) unsigned char pf_smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t full_bar[kPfStages], empty_bar[kPfStages], acc_bar;
+    unsigned char* bring = smem;
+    unsigned char* rring = bring + (size_t)kPfBStages * kPfBStageBytes;
+    float* xch = reinterpret_cast<float*>(rring + (size_t)kPfRawStages * kPfRawStageBytes);
+    int* s_dst = reinterpret_cast<int*>(xch + 2 * kPfXchFloats);
+    float* s_w = reinterpret_cast<float*>(s_dst + kPfMaxN);
+
+    __shared__ uint64_t raw_full[kPfRawStages], raw_empty[kPfRawStages], b_full[kPfBStages], b_empty[kPfBStages];
+    __shared__ uint64_t a_full[kPfAStages], a_empty[kPfAStages], acc_full[2], acc_empty[2], done_bar;
     __shared__ uint32_t tmem_base;
-    __shared__ int s_tok[kPfMaxN];
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_mtiles = kGemm1 ? (2 * a.NW) / 128 : a.NW / 128;
-    const int tile = blockIdx.x / n_mtiles, mt = blockIdx.x - tile * n_mtiles;
-    if (tile >= a.ctl[0]) return;  // uniform across the CTA
-    const int e = a.g_expert[tile], start = a.g_start[tile], count = a.g_count[tile];
-    const int N = (count + 15) & ~15;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_items = a.ctl[0] * a.n_mtiles;
     const int ksteps = a.K / kPfKStep;
+    const int rsteps = a.K / kPfRawK;
 
-    if (tid < kPfMaxN) s_tok[tid] = tid < count ? (kGemm1 ? a.pair_token[start + tid] : start + tid) : -1;
-    if (tid == 0) {
-        for (int s = 0; s < kPfStages; ++s) {
-            mbar_init(&full_bar[s], 2 * kPfProducers);  // per producer: A arrive + B arrive
-            mbar_init(&empty_bar[s], 1);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kPfRawStages; ++i) {
+            mbar_init(&raw_full[i], 1);
+            mbar_init(&raw_empty[i], 8);  // one arrival per dequant warp
         }
-        mbar_init(&acc_bar, 1);
+        for (int i = 0; i < kPfBStages; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
+        }
+        for (int i = 0; i < kPfAStages; ++i) {
+            mbar_init(&a_full[i], 8);
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+        }
+        mbar_init(&done_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 8) tmem_alloc(&tmem_base, kPfTmemCols);
+    if (warp == kPfWarpMma) tmem_alloc(&tmem_base, kPfTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
     const unsigned long long deadline = global_ns() + kPfWaitNs;
 
-    auto stage_a = [&](int s) { return smem + (size_t)s * kPfStageBytes; };
-    auto stage_b = [&](int s) { return smem + (size_t)s * kPfStageBytes + kPfABytes; };
-    auto stage_raw = [&](int r) { return smem + (size_t)kPfStages * kPfStageBytes + (size_t)r * kPfRawBytes; };
-
-    if (warp < 8) {
-        // ---------------- producers ----------------
-        const int row = tid >> 1, half = tid & 1;  // A: one 16-byte half-row of int4 per thread
-        // weight row of this thread in the tile
-        const uint8_t* qrow;
-        const float* srow;
-        if (kGemm1) {
-            // rows 0-31 gate n0.., 32-63 up n0.., 64-95 gate n0+32.., 96-127 up n0+32..
-            const int n = mt * 64 + (row >> 6) * 32 + (row & 31);
-            const bool up = (row >> 5) & 1;
-            const size_t r = (size_t)e * a.NW + n;
-            qrow = (up ? a.q1 : a.q0) + r * (a.K / 2);
-            srow = (up ? a.s1 : a.s0) + r * (a.K / kGroup);
-        } else {
-            const size_t r = (size_t)e * a.NW + mt * 128 + row;
-            qrow = a.q0 + r * (a.K / 2);
-            srow = a.s0 + r * (a.K / kGroup);
-        }
-        const size_t act_row_bytes = (size_t)a.K * ((kGemm1 && !kXBf16) ? 4 : 2);
-        bool ok = true;
-
-        // int4 bytes and scales of k-step ks -> raw ring slot ks % kPfRawStages (own data of this thread)
-        auto issue_raw = [&](int ks) {
-            unsigned char* raw = stage_raw(ks % kPfRawStages);
-            cp_async16(raw + row * 32 + half * 16, qrow + (size_t)ks * 32 + half * 16);
-            cp_async4(raw + 128 * 32 + (row * 2 + half) * 4, srow + ks);
-        };
-        // token rows of k-step ks -> MMA stage ks % kPfStages; the stage's full barrier gets
-        // this thread's arrival when its copies (and all earlier ones) have landed
-        auto issue_b = [&](int ks) {
-            const int s = ks % kPfStages;
-            if (kGemm1 && !kXBf16) return;  // fp32 activations: converted while storing, below
-            unsigned char* b = stage_b(s);
-            for (int i = tid; i < N * 8; i += kPfProducers) {
-                const int r = i >> 3, c = i & 7;
-                const int src_row = s_tok[r] >= 0 ? s_tok[r] : s_tok[0];
-                const unsigned char* src = static_cast<const unsigned char*>(a.act) + (size_t)src_row * act_row_bytes +
-                                           (size_t)ks * 128 + c * 16;
-                cp_async16(b + r * 128 + ((c ^ (r & 7)) * 16), src);
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            tma_prefetch_map(&tq0);
+            tma_prefetch_map(&tq1);
+            tma_prefetch_map(&ts0);
+            tma_prefetch_map(&ts1);
+            tma_prefetch_map(&tb);
+            int kb = 0, kr = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                const int tile = it / a.n_mtiles, mt = it - tile * a.n_mtiles;
+                const int e = a.g_expert[tile], start = a.g_start[tile], count = a.g_count[tile];
+                const int nbox = (count + kPfBRows - 1) / kPfBRows;
+                const int r0 = kGemm1 ? e * a.NW + mt * 64 : e * a.NW + mt * 128;
+                const int r1 = kGemm1 ? r0 : r0 + 64;
+                for (int j = 0; j < rsteps && ok; ++j) {
+                    const int sr = kr % kPfRawStages;
+                    if (kr >= kPfRawStages) ok = mbar_wait(&raw_empty[sr], ((kr / kPfRawStages) - 1) & 1, deadline, a.err);
+                    if (!ok) break;
+                    unsigned char* st = rring + (size_t)sr * kPfRawStageBytes;
+                    mbar_expect_tx(&raw_full[sr], kPfRawStageBytes);
+                    tma_load_2d(st, &tq0, j * (kPfRawK / 2), r0, &raw_full[sr]);
+                    tma_load_2d(st + kPfRawHalfBytes, &tq1, j * (kPfRawK / 2), r1, &raw_full[sr]);
+                    tma_load_2d(st + kPfRawScaleOff, &ts0, j * (kPfRawK / kGroup), r0, &raw_full[sr]);
+                    tma_load_2d(st + kPfRawScaleOff + 64 * 16, &ts1, j * (kPfRawK / kGroup), r1, &raw_full[sr]);
+                    ++kr;
+                    for (int s = 0; s < kPfRawK / kPfKStep; ++s) {
+                        const int sb = kb % kPfBStages;
+                        if (kb >= kPfBStages) ok = mbar_wait(&b_empty[sb], ((kb / kPfBStages) - 1) & 1, deadline, a.err);
+                        if (!ok) break;
+                        unsigned char* bs = bring + (size_t)sb * kPfBStageBytes;
+                        mbar_expect_tx(&b_full[sb], nbox * kPfBRows * 128);
+                        const int kx = (j * (kPfRawK / kPfKStep) + s) * kPfKStep;
+                        for (int i = 0; i < nbox; ++i)
+                            tma_load_2d(bs + i * kPfBRows * 128, &tb, kx, start + kPfBRows * i, &b_full[sb]);
+                        ++kb;
+                    }
+                }
             }
-        };
-
-        // prologue: int4 bytes kPfRawStages - 1 k-steps ahead, token rows kPfStages - 1 ahead
-        for (int ks = 0; ks < kPfRawStages - 1; ++ks) {
-            if (ks < ksteps) issue_raw(ks);
-            cp_async_commit();
+            // Let every issued copy land before the CTA can retire (normally long done).
+            const unsigned long long drain = global_ns() + kPfDrainNs;
+            for (int s = 0; s < kPfBStages && s < kb; ++s) {
+                const int last = kb - 1 - ((kb - 1 - s) % kPfBStages);
+                mbar_wait(&b_full[s], (last / kPfBStages) & 1, drain, a.err);
+            }
+            for (int s = 0; s < kPfRawStages && s < kr; ++s) {
+                const int last = kr - 1 - ((kr - 1 - s) % kPfRawStages);
+                mbar_wait(&raw_full[s], (last / kPfRawStages) & 1, drain, a.err);
+            }
         }
-        for (int ks = 0; ks < kPfStages - 1 && ks < ksteps; ++ks) {
-            issue_b(ks);
-            if (kGemm1 && !kXBf16) mbar_arrive(&full_bar[ks % kPfStages]);
-            else cp_async_arrive_noinc(&full_bar[ks % kPfStages]);
-        }
-        for (int ks = 0; ks < ksteps && ok; ++ks) {
-            const int s = ks % kPfStages;
-            // token rows for k-step ks + S - 1, once the MMA has released that stage
-            const int kb = ks + kPfStages - 1;
-            if (kb < ksteps) {
-                const int sb = kb % kPfStages, fill = kb / kPfStages;
-                if (fill > 0) ok = mbar_wait(&empty_bar[sb], (fill - 1) & 1, deadline, a.err);
+    } else if (warp == kPfWarpMma) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int kg = 0, kb = 0, local = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+                const int tile = it / a.n_mtiles;
+                const int N = (a.g_count[tile] + 15) & ~15;
+                const uint32_t idesc = idesc_bf16(N);
+                const int ab = local & 1, use = local >> 1;
+                if (use > 0) {
+                    ok = mbar_wait(&acc_empty[ab], (use - 1) & 1, deadline, a.err);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const uint32_t d = tmem + (uint32_t)(ab * kPfMaxN);
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int sa = kg % kPfAStages, sb = kb % kPfBStages;
+                    ok = mbar_wait(&a_full[sa], (kg / kPfAStages) & 1, deadline, a.err) &&
+                         mbar_wait(&b_full[sb], (kb / kPfBStages) & 1, deadline, a.err);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t bbase = smem_u32(bring + (size_t)sb * kPfBStageBytes);
+                    const uint32_t acol = tmem + (uint32_t)(kPfACol + sa * 32);
+#pragma unroll
+                    for (int kk = 0; kk < kPfKStep / 16; ++kk)
+                        tc_mma_ts(d, acol + kk * 8, smem_desc_sw128(bbase + kk * 32), idesc, (ks | kk) != 0);
+                    tc_commit(&a_empty[sa]);
+                    tc_commit(&b_empty[sb]);
+                    ++kg;
+                    ++kb;
+                }
                 if (!ok) break;
-                issue_b(kb);
-                if (kGemm1 && !kXBf16) mbar_arrive(&full_bar[sb]);
-                else cp_async_arrive_noinc(&full_bar[sb]);
+                tc_commit(&acc_full[ab]);
             }
-            // int4 bytes for k-step ks + R - 1 (its ring slot was consumed at k-step ks - 1)
-            if (ks + kPfRawStages - 1 < ksteps) issue_raw(ks + kPfRawStages - 1);
-            cp_async_commit();
-            cp_async_wait<kPfRawStages - 1>();  // the group of k-step ks has landed
-            unsigned char* raw = stage_raw(ks % kPfRawStages);
-            const uint4 w = *reinterpret_cast<const uint4*>(raw + row * 32 + half * 16);
-            const float sc = *reinterpret_cast<const float*>(raw + 128 * 32 + (row * 2 + half) * 4);
-            unsigned char* A = stage_a(s);
-            // q * s from the two mantissa windows (exact q; one fp32 rounding, then bf16)
-            const float s16 = 16.f * sc, m24 = -24.f * sc, s256 = 256.f * sc, m264 = -264.f * sc;
-            const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {  // 8 values per 16-byte chunk of the bf16 row
-                const uint32_t wd = words[c4], tt = wd >> 12;
-                const uint32_t sh[4] = {wd << 15, wd << 7, tt << 11, tt << 3};
-                uint32_t o[4];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 f = nib_pair(sh[p]);  // (odd k, even k) of the pair
-                    o[p] = bf16x2_of(fmaf(f.y, s256, m264), fmaf(f.x, s16, m24));
-                }
-                const int c = half * 4 + c4;
-                *reinterpret_cast<uint4*>(A + row * 128 + ((c ^ (row & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-            if (kGemm1 && !kXBf16) {
-                unsigned char* b = stage_b(s);
-                for (int i = tid; i < N * 8; i += kPfProducers) {
-                    const int r = i >> 3, c = i & 7;
-                    const int src_row = s_tok[r] >= 0 ? s_tok[r] : s_tok[0];
-                    const float* src = reinterpret_cast<const float*>(static_cast<const unsigned char*>(a.act) +
-                                                                      (size_t)src_row * act_row_bytes) +
-                                       (size_t)ks * 64 + c * 8;
-                    const float4 v0 = *reinterpret_cast<const float4*>(src);
-                    const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
-                    *reinterpret_cast<uint4*>(b + r * 128 + ((c ^ (r & 7)) * 16)) =
-                        make_uint4(bf16x2_of(v0.x, v0.y), bf16x2_of(v0.z, v0.w), bf16x2_of(v1.x, v1.y),
-                                   bf16x2_of(v1.z, v1.w));
-                }
-            }
-            fence_proxy_async();
-            mbar_arrive(&full_bar[s]);
+            tc_commit(&done_bar);  // every MMA issued above completes before TMEM is freed
         }
-        cp_async_wait<0>();
-
-        // ---------------- epilogue (warps 0-3: TMEM lane quadrants 0-3) ----------------
-        if (warp < 4) {
-            if (ok) ok = mbar_wait(&acc_bar, 0, deadline, a.err);
-            ok = __all_sync(0xFFFFFFFFu, ok);  // tcgen05.ld is warp-collective
+    } else if (warp < kPfWarpDeq) {
+        // ---------------- epilogue (warps 2-5: TMEM lane quadrants 2, 3, 0, 1) ----------------
+        const int qd = warp & 3, row = qd * 32 + lane, et = threadIdx.x - kPfWarpEpi * 32;
+        int local = 0;
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++local) {
+            const int tile = it / a.n_mtiles, mt = it - tile * a.n_mtiles;
+            const int start = a.g_start[tile], count = a.g_count[tile];
+            const int ab = local & 1;
+            if (!kGemm1) {
+                epi_bar();  // the previous item's readers are done with s_dst / s_w
+                for (int c = et; c < count; c += 128) {
+                    const int pos = start + c;
+                    int t, slot;
+                    if (pos < a.P) {
+                        const int pid = a.perm[pos];
+                        t = pid / a.k;
+                        slot = pid - t * a.k;
+                    } else {
+                        t = pos - a.P;
+                        slot = a.k;
+                    }
+                    s_dst[c] = t * (a.k + 1) + slot;
+                    s_w[c] = a.pair_w[pos];
+                }
+            }
+            const bool got = mbar_wait(&acc_full[ab], (local >> 1) & 1, deadline, a.err);
+            if (!epi_bar_and(__all_sync(0xFFFFFFFFu, got))) break;  // uniform over the 4 warps
             tc_fence_after();
-            float* stg = reinterpret_cast<float*>(stage_b(0));  // [128 rows][16 cols] fp32
-            for (int c0 = 0; c0 < N; c0 += 16) {
+            const uint32_t tacc = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(ab * kPfMaxN);
+            const int n16 = (count + 15) & ~15;
+            for (int c0 = 0, ch = 0; c0 < n16; c0 += 16, ++ch) {
                 float v[16];
-                if (ok) tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) stg[(warp * 32 + lane) * 17 + i] = ok ? v[i] : 0.f;
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                tmem_ld16(tacc + c0, v);
                 if (kGemm1) {
-                    // 64 outputs n x 16 tokens: thread -> (token c, 8 consecutive n)
-                    const int c = tid >> 3, nb = (tid & 7) * 8;
-                    if (c0 + c < count) {
-                        uint32_t o[4];
+                    float* xb = xch + (ch & 1) * kPfXchFloats;
+                    if (qd >= 2) {
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            float hv[2];
+                        for (int i = 0; i < 16; ++i) xb[(row - 64) * 17 + i] = v[i];
+                    }
+                    epi_bar();
+                    if (qd < 2) {
+                        const int fs = pf_store_pos(mt * 64 + row);
+                        uint16_t* hp = a.h + (size_t)(start + c0) * a.NW + fs;
 #pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const int nl = nb + 2 * p + q;                    // 0..63
-                                const int gr = (nl >> 5) * 64 + (nl & 31);        // gate row in the tile
-                                const float gv = stg[gr * 17 + c], uv = stg[(gr + 32) * 17 + c];
-                                hv[q] = gv / (1.0f + expf(-gv)) * uv;
+                        for (int i = 0; i < 16; ++i) {
+                            if (c0 + i < count) {
+                                const float g = v[i], u = xb[row * 17 + i];
+                                hp[(size_t)i * a.NW] = float_to_bf16_bits(g / (1.0f + expf(-g)) * u);
                             }
-                            o[p] = bf16x2_of(hv[0], hv[1]);
                         }
-                        const int pos = start + c0 + c;
-                        *reinterpret_cast<uint4*>(a.h + (size_t)pos * a.NW + mt * 64 + nb) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 } else {
-                    // 128 outputs n x 16 tokens: thread -> (token c of 8, 16 consecutive n), two passes
+                    uint16_t* yp = a.ys + mt * 128 + row;
 #pragma unroll
-                    for (int pass = 0; pass < 2; ++pass) {
-                        const int c = pass * 8 + (tid >> 4), nb = (tid & 15) * 8;
-                        if (c0 + c < count) {
-                            const int pos = start + c0 + c;
-                            int t, slot;
-                            if (pos < a.P) {
-                                const int pid = a.perm[pos];
-                                t = pid / a.k;
-                                slot = pid - t * a.k;
-                            } else {
-                                t = pos - a.P;
-                                slot = a.k;
-                            }
-                            const float wgt = a.pair_w[pos];
-                            uint32_t o[4];
-#pragma unroll
-                            for (int p = 0; p < 4; ++p)
-                                o[p] = bf16x2_of(wgt * stg[(nb + 2 * p) * 17 + c], wgt * stg[(nb + 2 * p + 1) * 17 + c]);
-                            *reinterpret_cast<uint4*>(a.ys + ((size_t)t * (a.k + 1) + slot) * a.NW + mt * 128 + nb) =
-                                make_uint4(o[0], o[1], o[2], o[3]);
-                        }
+                    for (int i = 0; i < 16; ++i) {
+                        if (c0 + i < count)
+                            yp[(size_t)s_dst[c0 + i] * a.NW] = float_to_bf16_bits(s_w[c0 + i] * v[i]);
                     }
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
             }
             tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
-    } else if (lane == 0) {
-        // ---------------- MMA issuer ----------------
-        const uint32_t idesc = idesc_bf16(N);
+    } else {
+        // ---------------- dequantise (warps 6-13) ----------------
+        const int qd = warp & 3, half = (warp - kPfWarpDeq) >> 2;
+        const int row = qd * 32 + lane, box = row >> 6, rr = row & 63;
+        const uint32_t tlane = (uint32_t)(qd * 32) << 16;
+        int kg = 0, kr = 0;
         bool ok = true;
-        for (int ks = 0; ks < ksteps; ++ks) {
-            const int s = ks % kPfStages;
-            ok = mbar_wait(&full_bar[s], (ks / kPfStages) & 1, deadline, a.err);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t abase = smem_u32(stage_a(s)), bbase = smem_u32(stage_b(s));
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc_mma(tmem, smem_desc_sw128(abase + kk * 32), smem_desc_sw128(bbase + kk * 32), idesc,
-                       (ks | kk) != 0);
-            tc_commit(&empty_bar[s]);
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            for (int ks = 0; ks < ksteps; ++ks) {
+                const int sub = ks % (kPfRawK / kPfKStep), sr = kr % kPfRawStages, sa = kg % kPfAStages;
+                if (sub == 0) ok = mbar_wait(&raw_full[sr], (kr / kPfRawStages) & 1, deadline, a.err);
+                if (ok && kg >= kPfAStages) ok = mbar_wait(&a_empty[sa], ((kg / kPfAStages) - 1) & 1, deadline, a.err);
+                ok = __all_sync(0xFFFFFFFFu, ok);
+                if (!ok) break;
+                const unsigned char* st = rring + (size_t)sr * kPfRawStageBytes;
+                const int c = sub * 2 + half;  // 16-byte chunk of the 128-byte row
+                const uint4 w =
+                    *reinterpret_cast<const uint4*>(st + box * kPfRawHalfBytes + rr * 128 + ((c ^ (rr & 7)) << 4));
+                const float s = *reinterpret_cast<const float*>(st + kPfRawScaleOff + box * 64 * 16 + rr * 16 + sub * 4);
+                if (sub == kPfRawK / kPfKStep - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&raw_empty[sr]);
+                    ++kr;
+                }
+                uint32_t o[16];
+                dequant32(w, s, o);
+                tc_fence_after();
+                tmem_st16(tmem + tlane + (uint32_t)(kPfACol + sa * 32 + half * 16), o);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[sa]);
+                ++kg;
+            }
         }
-        tc_commit(&acc_bar);  // also on a timeout: every issued MMA completes before TMEM is freed
     }
+
     __syncthreads();
-    tc_fence_after();
-    if (warp == 8) {
-        if (lane == 0) mbar_wait(&acc_bar, 0, deadline, a.err);
+    if (warp == kPfWarpMma) {
+        if (lane == 0) mbar_wait(&done_bar, 0, global_ns() + kPfDrainNs, a.err);
         __syncwarp();
+        tc_fence_after();
         tmem_dealloc(tmem, kPfTmemCols);
     }
+}
+
+// Token rows of every sorted position, bf16, in the permuted K order:
+// xg[pos, 8g + p] = x[pair_token[pos], 8g + sigma(p)].
+template <bool kXBf16>
+__global__ void prefill_gather_kernel(const void* __restrict__ x, const int32_t* __restrict__ pair_token, int Q,
+                                      int H, uint16_t* __restrict__ xg)
+{
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int g8 = H / 8;
+    if (i >= (size_t)Q * g8) return;
+    const int pos = (int)(i / g8), g = (int)(i - (size_t)pos * g8);
+    const int t = pair_token[pos];
+    float v[8];
+    if constexpr (kXBf16) {
+        const uint4 r = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)t * H + 8 * g);
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[2 * j] = bf16_bits_to_float(w[j] & 0xFFFFu);
+            v[2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
+        }
+    } else {
+        const float* src = static_cast<const float*>(x) + (size_t)t * H + 8 * g;
+        const float4 a0 = *reinterpret_cast<const float4*>(src), a1 = *reinterpret_cast<const float4*>(src + 4);
+        v[0] = a0.x, v[1] = a0.y, v[2] = a0.z, v[3] = a0.w, v[4] = a1.x, v[5] = a1.y, v[6] = a1.z, v[7] = a1.w;
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+        o[m] = (uint32_t)float_to_bf16_bits(v[m]) | ((uint32_t)float_to_bf16_bits(v[m + 4]) << 16);
+    *reinterpret_cast<uint4*>(xg + (size_t)pos * H + 8 * g) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // out[t, n] = sum over slots j (routed in slot order, shared last) of ys[t, j, n].

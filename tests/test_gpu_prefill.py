@@ -45,9 +45,11 @@ def _tie_free(rng, T, H, w_router, sel_bias, k, alpha, bf16):
 
 
 @pytest.mark.parametrize("H,F,E,k,T,xdt,odt", [
-    (256, 128, 16, 4, 100, "bf16", "f32"),
-    (256, 128, 16, 4, 300, "f32", "bf16"),
+    (256, 256, 16, 4, 100, "bf16", "f32"),
+    (256, 256, 16, 4, 300, "f32", "bf16"),
     (1024, 512, 64, 8, 520, "bf16", "bf16"),
+    # 250 pairs per routed expert: every expert spans two token tiles (ragged second tile)
+    (512, 256, 8, 2, 1000, "bf16", "bf16"),
 ])
 def test_prefill_matches_oracle(env, H, F, E, k, T, xdt, odt):
     coli, torch = env
