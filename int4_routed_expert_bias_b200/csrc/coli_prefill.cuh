@@ -13,8 +13,8 @@
 //   warp 0     TMA producer: int4 bytes + scales of the weight tile, 256 K at a
 //              time (3-deep ring), and the token rows (bf16), 64 K at a time
 //              (5-deep ring), straight into the 128-byte-swizzled layouts;
-//   warps 6-13 dequantise: each thread owns one weight row (= TMEM lane) and
-//              half of a 64-K step; q * s is formed in bf16 and written into a
+//   warps 6..  dequantise: each thread owns one weight row (= TMEM lane) and
+//              a part of a 64-K step; q * s is formed in bf16 and written into a
 //              4-deep ring of A operands in TMEM with tcgen05.st;
 //   warp 1     one thread issues tcgen05.mma (A from TMEM, B from shared memory,
 //              M 128, K 16, fp32 accumulate) into one of two TMEM accumulators;
@@ -54,14 +54,21 @@ constexpr int kPfRawHalfBytes = 64 * kPfRawK / 2;             // int4 bytes of 6
 constexpr int kPfRawScaleOff = 2 * kPfRawHalfBytes;          // then 2 x 64 rows x 4 scales
 constexpr int kPfRawStageBytes = kPfRawScaleOff + 2 * 64 * 16;
 constexpr int kPfXchFloats = 64 * 17;                        // gate/up exchange, one buffer
-constexpr int kPfThreads = 14 * 32;
-constexpr int kPfWarpMma = 1, kPfWarpEpi = 2, kPfWarpDeq = 6;
+#ifndef COLI_PF_DEQ_WARPS
+#define COLI_PF_DEQ_WARPS 8
+#endif
+constexpr int kPfDeqWarps = COLI_PF_DEQ_WARPS;   // 8 or 16: each takes 64 / (warps / 4) K of a step
+constexpr int kPfDeqParts = kPfDeqWarps / 4;     // warps per TMEM lane quadrant
+constexpr int kPfDeqK = kPfKStep / kPfDeqParts;  // K values per dequant thread per step
+constexpr int kPfWarpMma = 1, kPfWarpEpi = 2, kPfWarpDeq = 6, kPfWarpEnd = 6 + kPfDeqWarps;
+constexpr int kPfThreads = kPfWarpEnd * 32;
 constexpr size_t kPfSmemBytes = 1024 /*alignment slack*/ + (size_t)kPfBStages * kPfBStageBytes +
                                 (size_t)kPfRawStages * kPfRawStageBytes + 2 * kPfXchFloats * 4 + 2 * kPfMaxN * 4;
 constexpr unsigned long long kPfWaitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr unsigned long long kPfDrainNs = 100000000ull;  // teardown waits
 
 static_assert(kPfACol + kPfAStages * 32 <= kPfTmemCols, "TMEM budget");
+static_assert(kPfDeqWarps == 8 || kPfDeqWarps == 16, "dequant split");
 static_assert(kPfMaxN % kPfBRows == 0 && kPfMaxN % 16 == 0 && kPfMaxN <= 256, "tile width");
 static_assert(kPfBStageBytes % 1024 == 0 && kPfRawStageBytes % 1024 == 0, "swizzled stages stay 1024-aligned");
 
@@ -107,12 +114,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// Same, but the thread may be suspended (issuing nothing) until the phase
+// completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; false after the
-// deadline (error word set).
+// deadline (error word set).  Waiting threads sleep in the barrier instead of
+// spinning, so they take no issue slots from the warps doing the work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long deadline, int* err)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, 1000000u)) {
         if (global_ns() > deadline) {
             atomicExch(err, 1);
             return false;
@@ -197,17 +220,26 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Store 16 consecutive 32-bit TMEM columns of this thread's lane and wait for them.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+// Store NC (8 or 16) consecutive 32-bit TMEM columns of this thread's lane
+// (asynchronous: tmem_wait_st() waits for all of this thread's stores).
+template <int NC>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[NC])
 {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    if constexpr (NC == 16) {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::
+                "r"(taddr),
+            "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+            "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+            : "memory");
+    } else {
+        static_assert(NC == 8, "8 or 16 columns");
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                     "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                     : "memory");
+    }
 }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, rows of 128 bytes,
 // 8-row groups 1024 bytes apart (tcgen05 descriptor version 1).
@@ -230,18 +262,18 @@ __device__ __forceinline__ uint32_t idesc_bf16(int n)
 
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
-// 32 int4 weights (16 bytes, low nibble first) of one row -> 16 bf16x2 words of
-// q * s.  Word 4i + m holds (nibble m, nibble m + 4) of 32-bit word i: the mask
-// picks bits 0-3 and 16-19 after a shift by 4m, and the xor makes each half the
-// bf16 number 128 + (nibble ^ 8) = 136 + q (exponent 2^7: one unit per step).
-// q = v - 136 is exact; q * bf16(s) is rounded once to bf16.
-__device__ __forceinline__ void dequant32(uint4 w, float s, uint32_t (&o)[16])
+// 8 * NW int4 weights (NW 32-bit words, low nibble first) of one row -> 4 * NW
+// bf16x2 words of q * s.  Word 4i + m holds (nibble m, nibble m + 4) of 32-bit
+// word i: the mask picks bits 0-3 and 16-19 after a shift by 4m, and the xor
+// makes each half the bf16 number 128 + (nibble ^ 8) = 136 + q (exponent 2^7:
+// one unit per step).  q = v - 136 is exact; q * bf16(s) is rounded once to bf16.
+template <int NW>
+__device__ __forceinline__ void dequant_words(const uint32_t (&words)[NW], float s, uint32_t (&o)[4 * NW])
 {
     const __nv_bfloat162 s2 = __float2bfloat162_rn(s);
     const __nv_bfloat162 c136 = __float2bfloat162_rn(136.f);
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < NW; ++i) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             uint32_t v;
@@ -306,14 +338,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap tq0, const __grid_consta
     if (threadIdx.x == 0) {
         for (int i = 0; i < kPfRawStages; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], 8);  // one arrival per dequant warp
+            mbar_init(&raw_empty[i], kPfDeqWarps);  // one arrival per dequant warp
         }
         for (int i = 0; i < kPfBStages; ++i) {
             mbar_init(&b_full[i], 1);
             mbar_init(&b_empty[i], 1);
         }
         for (int i = 0; i < kPfAStages; ++i) {
-            mbar_init(&a_full[i], 8);
+            mbar_init(&a_full[i], kPfDeqWarps);
             mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -482,39 +514,64 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap tq0, const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
-    } else {
-        // ---------------- dequantise (warps 6-13) ----------------
-        const int qd = warp & 3, half = (warp - kPfWarpDeq) >> 2;
+    } else if (warp < kPfWarpEnd) {
+        // ---------------- dequantise (warps 6 ..) ----------------
+        // One flat sequence over this CTA's k-steps (K is a multiple of the int4
+        // stage, so stage boundaries line up with items).  Software-pipelined:
+        // the TMEM store of step n is in flight while step n + 1 is read and
+        // dequantised.
+        constexpr int kWords = kPfDeqK / 8;  // 32-bit words of int4 per thread and step
+        constexpr int kSubs = kPfRawK / kPfKStep;
+        const int qd = warp & 3, part = (warp - kPfWarpDeq) >> 2;
         const int row = qd * 32 + lane, box = row >> 6, rr = row & 63;
         const uint32_t tlane = (uint32_t)(qd * 32) << 16;
-        int kg = 0, kr = 0;
-        bool ok = true;
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            for (int ks = 0; ks < ksteps; ++ks) {
-                const int sub = ks % (kPfRawK / kPfKStep), sr = kr % kPfRawStages, sa = kg % kPfAStages;
-                if (sub == 0) ok = mbar_wait(&raw_full[sr], (kr / kPfRawStages) & 1, deadline, a.err);
-                if (ok && kg >= kPfAStages) ok = mbar_wait(&a_empty[sa], ((kg / kPfAStages) - 1) & 1, deadline, a.err);
-                ok = __all_sync(0xFFFFFFFFu, ok);
-                if (!ok) break;
-                const unsigned char* st = rring + (size_t)sr * kPfRawStageBytes;
-                const int c = sub * 2 + half;  // 16-byte chunk of the 128-byte row
-                const uint4 w =
-                    *reinterpret_cast<const uint4*>(st + box * kPfRawHalfBytes + rr * 128 + ((c ^ (rr & 7)) << 4));
-                const float s = *reinterpret_cast<const float*>(st + kPfRawScaleOff + box * 64 * 16 + rr * 16 + sub * 4);
-                if (sub == kPfRawK / kPfKStep - 1) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&raw_empty[sr]);
-                    ++kr;
-                }
-                uint32_t o[16];
-                dequant32(w, s, o);
-                tc_fence_after();
-                tmem_st16(tmem + tlane + (uint32_t)(kPfACol + sa * 32 + half * 16), o);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[sa]);
-                ++kg;
+        const int my_items = n_items > (int)blockIdx.x ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+        const int total = my_items * ksteps;
+        uint32_t words[kWords];
+        float scale = 0.f;
+        // int4 words and scale of step n (waits for its stage; frees the stage after its last step)
+        auto load = [&](int n) -> bool {
+            const int sub = n % kSubs, kr = n / kSubs, sr = kr % kPfRawStages;
+            bool ok = true;
+            if (sub == 0) ok = mbar_wait(&raw_full[sr], (kr / kPfRawStages) & 1, deadline, a.err);
+            if (!__all_sync(0xFFFFFFFFu, ok)) return false;
+            const unsigned char* st = rring + (size_t)sr * kPfRawStageBytes;
+            // this thread's bytes: K [sub * 64 + part * kPfDeqK, + kPfDeqK) of the stage
+            const int byte0 = sub * 32 + part * (kPfDeqK / 2);
+            const int c = byte0 >> 4;  // 16-byte chunk of the 128-byte row
+            const unsigned char* src = st + box * kPfRawHalfBytes + rr * 128 + ((c ^ (rr & 7)) << 4) + (byte0 & 15);
+            if constexpr (kWords == 4) {
+                const uint4 w = *reinterpret_cast<const uint4*>(src);
+                words[0] = w.x, words[1] = w.y, words[2] = w.z, words[3] = w.w;
+            } else {
+                const uint2 w = *reinterpret_cast<const uint2*>(src);
+                words[0] = w.x, words[1] = w.y;
             }
+            scale = *reinterpret_cast<const float*>(st + kPfRawScaleOff + box * 64 * 16 + rr * 16 + sub * 4);
+            if (sub == kSubs - 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&raw_empty[sr]);
+            }
+            return true;
+        };
+        uint32_t o[4 * kWords];
+        bool ok = total > 0 && load(0);
+        if (ok) dequant_words<kWords>(words, scale, o);
+        for (int n = 0; n < total && ok; ++n) {
+            const int sa = n % kPfAStages;
+            bool got = true;
+            if (n >= kPfAStages) got = mbar_wait(&a_empty[sa], ((n / kPfAStages) - 1) & 1, deadline, a.err);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            tc_fence_after();
+            tmem_st<4 * kWords>(tmem + tlane + (uint32_t)(kPfACol + sa * 32 + part * (kPfDeqK / 2)), o);
+            if (n + 1 < total) {
+                ok = load(n + 1);
+                if (ok) dequant_words<kWords>(words, scale, o);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[sa]);
         }
     }
 
