@@ -89,7 +89,7 @@ coli_status device_info(DeviceInfo** out)
         if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
             (e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
             return cuda_fail(e, "cudaDeviceGetAttribute");
-        const int lim = d.smem_optin - 1024;  // room for the kernels' static shared memory
+        const int lim = d.smem_optin - 8192;  // room for the kernels' static shared memory
         if ((e = allow_smem(expert_phase_kernel<true, false, 1>, lim)) != cudaSuccess ||
             (e = allow_smem(expert_phase_kernel<true, false, 4>, lim)) != cudaSuccess ||
             (e = allow_smem(expert_phase_kernel<true, true, 1>, lim)) != cudaSuccess ||
