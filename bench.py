@@ -147,12 +147,20 @@ def dist_env():
 
 
 def max_over_ranks(value, world, torch):
+    """The largest `value` over all ranks (every rank gets it)."""
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, steps, tokens_per_step, ms_max):
+    """Whole-job tokens/s: each of `world` ranks ran `steps` layer calls of
+    `tokens_per_step` tokens, and the job lasted as long as its slowest rank."""
+    return world * steps * tokens_per_step / (ms_max * 1e-3)
 
 
 def barrier(world):
@@ -362,7 +370,7 @@ def run_ours(args):
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms, world, torch)
     ms_per_step = ms_max / steps
-    value = world * steps * c.T / (ms_max * 1e-3)
+    value = job_throughput(world, steps, c.T, ms_max)
 
     # stage timings of the last G calls (inside the timed region)
     stage_ms = {n: float(np.mean([ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]) for i in range(G)]))
@@ -429,7 +437,7 @@ def run_ours(args):
         e1.record(s)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world, torch)
-        line["e2e"] = {"value": world * n_e2e * c.T / (ems * 1e-3), "unit": "tokens/s",
+        line["e2e"] = {"value": job_throughput(world, n_e2e, c.T, ems), "unit": "tokens/s",
                        "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
                        "steps": n_e2e, "host_sync_per_step": True}
 
