@@ -34,12 +34,12 @@ STAGE_NAMES = ("route", "union", "gateup", "down", "combine")
 
 
 def kernels_per_call(T, E):
-    """Our kernel launches in one layer call: batch 1 runs router scores, gate/up
-    (with top-k), down and combine; decode batches run router scores, top-k +
+    """Our kernel launches in one layer call: batch 1 runs router scores, top-k,
+    gate/up, down and combine; decode batches run router scores, top-k +
     union (one kernel up to 256 tokens), gate/up, down and combine; prefill
     batches add the token-row gather in front of the two grouped GEMMs."""
     if T == 1:
-        return 4
+        return 5
     fused = T <= 256 and E <= 256
     if T <= 64:
         return 5 if fused else 6

@@ -400,15 +400,18 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     float* wt = topk_w_out ? topk_w_out : w.w;
     const bool bf16 = (xt == COLI_BF16);
 
-    // One token: router scores, then gate/up (top-k in every CTA), then down with
-    // the combine fused; the union of a one-token batch is its k experts.
+    // One token: router scores, top-k, gate/up, down, combine; the union of a
+    // one-token batch is its k experts.
     const size_t s1_gu = stage_smem_bytes(H, 1), s1_dn = stage_smem_bytes(F, k + 1);
-    // (batch-1 path: router scores, gate/up, down, combine; see coli_decode1.cuh)
+    // (batch-1 path: see coli_decode1.cuh)
     if (T == 1 && E <= 256 && H == 1024 * 2 * kHalf && F == 2048 &&
         s1_gu <= (size_t)dev->smem_optin && s1_dn <= (size_t)dev->smem_optin) {
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
         st = launch_logits(x, xt, 1, H, L->w_router, E, w.logits, nullptr, 0, stream);
         if (st != COLI_OK) return st;
+        if ((e = launch_pdl(router_topk_kernel, 1, 32, 0, stream, (const float*)w.logits, 1, E, k, L->sel_bias,
+                            L->routed_scale, idx, wt)) != cudaSuccess)
+            return cuda_fail(e, "top-k launch");
         if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess ||
             (e = tm.rec(COLI_STAGE_UNION, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_GATEUP, 0)) != cudaSuccess)
             return cuda_fail(e, "event record");

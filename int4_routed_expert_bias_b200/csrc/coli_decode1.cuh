@@ -1,11 +1,11 @@
-// coli_decode1.cuh -- the layer for one token (batch-1 decode), four launches:
-//   router scores (router_logits_kernel, also zeroes the work counters)
-//   gateup_single_kernel:  top-k (every CTA, from the router scores), then
-//                          h_j = silu(W_gate,e_j x) * (W_up,e_j x) for the k
+// coli_decode1.cuh -- the layer for one token (batch-1 decode), five launches:
+//   router scores (router_logits_kernel)
+//   router_topk_kernel:    top-k of the scores, one warp
+//   gateup_single_kernel:  h_j = silu(W_gate,e_j x) * (W_up,e_j x) for the k
 //                          selected experts and the shared expert
 //   down_single_kernel:    partial_j = w_j W_down,e_j h_j (w = 1 for shared)
 //   combine_single_kernel: out = sum_j partial_j in slot order (deterministic)
-// The last three are launched as programmatic dependents of their predecessor,
+// The last four are launched as programmatic dependents of their predecessor,
 // so their launch overlaps its tail; they wait (griddepcontrol.wait) before
 // reading its results.
 //
@@ -86,17 +86,14 @@ __device__ __forceinline__ void half_compute(const float4* xs, const float* corr
 // keeps the integer pipe busy, so the kernel relies on occupancy (32 warps per
 // SM at <= 64 registers) to keep loads in flight; each half-row's loads are
 // issued together.  A warp whose first unit is a shared-expert row issues its
-// loads before the router's top-k is known; the staging of x and warp 0's
-// top-k overlap them.  kPL = chunks per lane = H / 1024 (two halves of kHalf).
+// loads before the routing is known; the staging of x and the wait for the
+// routing overlap them.  kPL = chunks per lane = H / 1024 (two halves of kHalf).
 template <bool kBf16>
 __global__ void __launch_bounds__(kSingleThreads, 2)
 gateup_single_kernel(SingleArgs a)
 {
     constexpr int kPL = 2 * kHalf;
     extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int s_e[kMaxTopK + 1];
-    __shared__ int32_t s_idx[kMaxTopK];
-    __shared__ float s_w[kMaxTopK];
     const StageGeom g = stage_geom(a.H);  // g.per_lane == kPL on this path
     float4* xs = reinterpret_cast<float4*>(smem);
     float* corr = reinterpret_cast<float*>(smem + (size_t)g.f4 * 16);
@@ -124,19 +121,9 @@ gateup_single_kernel(SingleArgs a)
         half_load<0>(gq, uq, gs, us, A);
     }
     stage_vectors<kBf16>(a.x, a.H, 1, [](int) { return 0; }, g, xs, corr);  // x is this call's input
-    griddep_wait();  // router scores of this call are complete
-    if (warp == 0) {
-        topk_warp_t<8>(a.logits, a.E, a.k, a.sel_bias, a.routed_scale, s_idx, s_w);  // E <= 256 on this path
-        __syncwarp();
-        if (lane < a.k) {
-            s_e[lane] = s_idx[lane];
-            if (blockIdx.x == 0) {
-                a.idx[lane] = s_idx[lane];
-                a.w[lane] = s_w[lane];
-            }
-        }
-    }
     __syncthreads();
+    griddep_wait();  // the routing of this call (router_topk_kernel) is complete
+    const int my_e = lane < a.k ? a.idx[lane] : a.E;  // expert of routed slot j + 1 in lane j
 
     bool loaded = first_shared;
     int sl = u / a.F, n = u - sl * a.F;  // slot index (0 = shared) and row of unit u
@@ -144,7 +131,8 @@ gateup_single_kernel(SingleArgs a)
     while (sl <= a.k) {
         const uint8_t *gq, *uq;
         const float *gs, *us;
-        rows(sl == 0 ? a.E : s_e[sl - 1], n, gq, uq, gs, us);
+        const int er = __shfl_sync(0xFFFFFFFFu, my_e, sl > 0 ? sl - 1 : 0);  // sl is warp-uniform
+        rows(sl == 0 ? a.E : er, n, gq, uq, gs, us);
         float tg = 0.f, tu = 0.f;
         if (!loaded) half_load<0>(gq, uq, gs, us, A);
         loaded = false;

@@ -191,102 +191,73 @@ __device__ __forceinline__ void topk_warp_rounds(const float* lrow, int E, int k
     }
 }
 
-// Top-k of one token by one warp for E <= 32 * kPer with few experts per lane
-// (same result as topk_warp_rounds, far shorter dependency chain):
-//   1. key of each expert: c = sigmoid(logit) + bias (NaN -> -inf, -0 -> +0),
-//      mapped to an unsigned integer with the same order;
-//   2. the k-th largest key T by a bitwise search, one warp-wide count per bit;
-//   3. winners: keys above T, then keys equal to T in ascending expert index;
-//   4. each winner's position = number of winners ahead of it in (c desc,
-//      index asc) order.
-// Weights are renormalised over the winners' sigmoids summed in position order.
+// Top-k of one token by one warp for E <= 32 * kPer (same result as
+// topk_warp_rounds, shorter dependency chain): every candidate gets one 64-bit
+// key, high word an order-preserving image of c = sigmoid(logit) + bias (NaN ->
+// -inf, -0 -> +0), low word the complement of the expert index, so a larger key
+// means (c desc, index asc) and keys are unique.  Each lane sorts its kPer keys;
+// then k rounds take the warp-wide maximum of the lanes' heads, and the lane
+// that owns it pops its head.
 template <int kPer>
-__device__ __forceinline__ void topk_warp_radix(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
+__device__ __forceinline__ void topk_warp_heads(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
                                                 float routed_scale, int32_t* idx_row, float* w_row)
 {
     const int lane = threadIdx.x & 31;
-    float s[kPer], c[kPer];
-    uint32_t m[kPer];  // order-preserving key; 0 = no expert (below every real key)
+    unsigned long long key[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
+        key[i] = 0ull;  // no expert: below every real key
         if (e < E) {
-            const float l = lrow[e];
-            s[i] = 1.0f / (1.0f + expf(-l));
-            const float ci = s[i] + sel_bias[e];
-            c[i] = (ci == ci) ? ci + 0.0f : -INFINITY;  // NaN ranks last; -0 and +0 are one key
-            const uint32_t u = __float_as_uint(c[i]);
-            m[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-        } else {
-            s[i] = 0.f;
-            c[i] = -INFINITY;
-            m[i] = 0u;
+            const float s = 1.0f / (1.0f + expf(-lrow[e]));
+            const float ci = s + sel_bias[e];
+            const float c = (ci == ci) ? ci + 0.0f : -INFINITY;
+            const uint32_t u = __float_as_uint(c);
+            const uint32_t m = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+            key[i] = ((unsigned long long)m << 32) | (uint32_t)(0xFFFFu - e);
         }
     }
-    // 2. k-th largest key: the largest T with at least k keys >= T
-    uint32_t T = 0u;
-#pragma unroll 1
-    for (int b = 31; b >= 0; --b) {
-        const uint32_t cand = T | (1u << b);
-        uint32_t cnt = 0;
+    // descending sort of the lane's keys (odd-even transposition; kPer is small)
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) cnt += m[i] >= cand ? 1u : 0u;
-        if (__reduce_add_sync(0xFFFFFFFFu, cnt) >= (uint32_t)k) T = cand;
-    }
-    // 3. winners
-    uint32_t above = 0;
+    for (int r = 0; r < kPer; ++r)
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) above += m[i] > T ? 1u : 0u;
-    int need = k - (int)__reduce_add_sync(0xFFFFFFFFu, above);  // ties to take, lowest index first
-    const uint32_t lt = (1u << lane) - 1u;
-    uint32_t sel = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        const bool tie = m[i] == T;
-        const uint32_t bt = __ballot_sync(0xFFFFFFFFu, tie);
-        if (m[i] > T || (tie && __popc(bt & lt) < need)) sel |= 1u << i;
-        need -= min(need, __popc(bt));
-    }
-    // 4. positions
-    int pos[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) pos[i] = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        uint32_t bw = __ballot_sync(0xFFFFFFFFu, (sel >> i) & 1u);
-        while (bw) {
-            const int src = __ffs(bw) - 1;
-            bw &= bw - 1;
-            const float oc = __shfl_sync(0xFFFFFFFFu, c[i], src);
-            const int oe = src + 32 * i;
-#pragma unroll
-            for (int i2 = 0; i2 < kPer; ++i2) {
-                const int me = lane + 32 * i2;
-                pos[i2] += (oc > c[i2] || (oc == c[i2] && oe < me)) ? 1 : 0;
-            }
+        for (int i = r & 1; i + 1 < kPer; i += 2) {
+            const unsigned long long a = key[i], b = key[i + 1];
+            key[i] = a > b ? a : b;
+            key[i + 1] = a > b ? b : a;
         }
-    }
+    unsigned long long mine = 0ull;  // lane j: the j-th winner
+    for (int j = 0; j < k; ++j) {
+        unsigned long long best = key[0];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i)
-        if ((sel >> i) & 1u) {
-            idx_row[pos[i]] = lane + 32 * i;
-            w_row[pos[i]] = s[i];
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+            best = other > best ? other : best;
         }
-    __syncwarp();
-    const float my_s = lane < k ? w_row[lane] : 0.f;
+        if (key[0] == best) {  // unique owner pops its head
+#pragma unroll
+            for (int i = 0; i + 1 < kPer; ++i) key[i] = key[i + 1];
+            key[kPer - 1] = 0ull;
+        }
+        if (lane == j) mine = best;
+    }
+    const int my_e = (int)(0xFFFFu - (uint32_t)(mine & 0xFFFFu));
+    const float my_s = lane < k ? 1.0f / (1.0f + expf(-lrow[my_e])) : 0.f;
     float total = 0.f;
     for (int j = 0; j < k; ++j) total += __shfl_sync(0xFFFFFFFFu, my_s, j);
-    __syncwarp();
-    if (lane < k) w_row[lane] = routed_scale * my_s / total;
+    if (lane < k) {
+        idx_row[lane] = my_e;
+        w_row[lane] = routed_scale * my_s / total;
+    }
 }
 
-// Default warp top-k: the bitwise search for up to 8 experts per lane, rounds of
-// arg-max above that.
+// Default warp top-k: the tournament of sorted heads for up to 8 experts per
+// lane, rounds of arg-max above that.
 template <int kPer>
 __device__ __forceinline__ void topk_warp_t(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
                                             float routed_scale, int32_t* idx_row, float* w_row)
 {
-    if constexpr (kPer <= 8) topk_warp_radix<kPer>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
+    if constexpr (kPer <= 8) topk_warp_heads<kPer>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
     else topk_warp_rounds<kPer>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
 }
 
@@ -297,12 +268,16 @@ __device__ __forceinline__ void topk_warp(const float* lrow, int E, int k, const
     else topk_warp_t<kMaxExperts / 32>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
 }
 
-// One warp per token, logits from global memory (layer path).
+// One warp per token, logits from global memory (layer path).  When launched as
+// a programmatic dependent it waits for the router scores, and lets its own
+// dependent launch at once (that kernel waits for this one's results).
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                    const float* __restrict__ sel_bias, float routed_scale,
                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;  // whole warp leaves together
     topk_warp(logits + (size_t)t * E, E, k, sel_bias, routed_scale, topk_idx + (size_t)t * k,
