@@ -402,7 +402,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
 
     // One token: router scores, top-k, gate/up, down, combine; the union of a
     // one-token batch is its k experts.
-    const size_t s1_gu = stage_smem_bytes(H, 1), s1_dn = stage_smem_bytes(F, k + 1);
+    const size_t s1_gu = stage_smem_bytes(H, 1), s1_dn = stage_smem_bytes(F, 1);
     // (batch-1 path: see coli_decode1.cuh)
     if (T == 1 && E <= 256 && H == 1024 * 2 * kHalf && F == 2048 &&
         s1_gu <= (size_t)dev->smem_optin && s1_dn <= (size_t)dev->smem_optin) {
@@ -427,7 +427,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
             return cuda_fail(e, "event record");
         {
             auto kern = down_single_kernel<0>;
-            if ((e = launch_pdl(kern, dev->sms * blocks_per_sm(kern, s1_dn, kSingleThreads), kSingleThreads, s1_dn,
+            if ((e = launch_pdl(kern, std::max(dev->sms * blocks_per_sm(kern, s1_dn, kSingleThreads), k + 1), kSingleThreads, s1_dn,
                                 stream, sa)) != cudaSuccess)
                 return cuda_fail(e, "down launch");
         }

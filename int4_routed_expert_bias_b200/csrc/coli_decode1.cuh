@@ -193,58 +193,48 @@ __device__ __forceinline__ void down_compute(const float4* hs_j, const float* co
 
 // One work unit = (slot j, output rows n, n+1): partial[j][n..n+1] =
 // w_j * (W_down,e_j h_j)[n..n+1] (w = 1 for the shared expert).  The two rows
-// share every staged h load.  Units run row-pair-major (the k+1 slots of a row
-// pair are neighbours) and are dealt out statically; the next unit's loads are
-// issued before this unit's reduction.  combine_single_kernel then sums the
-// partials in slot order (deterministic).
+// share every staged h load.  Each CTA serves one slot (CTA b takes slot
+// b mod (k+1)), so it stages only that slot's h after the gate/up kernel is
+// done; the slot's row pairs are dealt out statically over its CTAs' warps, and
+// the next unit's loads are issued before this unit's reduction.
+// combine_single_kernel then sums the partials in slot order (deterministic).
 template <int kUnused = 0>
 __global__ void __launch_bounds__(kSingleThreads, 2)
 down_single_kernel(SingleArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ int s_e[kMaxTopK + 1];
-    __shared__ float s_w[kMaxTopK + 1];
     const int S = a.k + 1;  // slots: k routed + shared
     const StageGeom g = stage_geom(a.F);  // g.per_lane == 2 on this path
     float4* hs = reinterpret_cast<float4*>(smem);
-    float* corr = reinterpret_cast<float*>(smem + (size_t)S * g.f4 * 16);
+    float* corr = reinterpret_cast<float*>(smem + (size_t)g.f4 * 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int W = gridDim.x * kSingleWarps;
-    const int units = (a.H / 2) * S;
+    const int j = blockIdx.x % S;                           // this CTA's slot
+    const int nc = ((int)gridDim.x - j + S - 1) / S;        // CTAs serving slot j
+    const int Wj = nc * kSingleWarps;                        // their warps
+    const int pairs = a.H / 2;
     int off[8];
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) off[jj] = jj * 32 + (lane ^ jj);
 
     griddep_wait();  // routing and h of this call are complete
-    if (threadIdx.x < S) {
-        s_e[threadIdx.x] = threadIdx.x < a.k ? a.idx[threadIdx.x] : a.E;
-        s_w[threadIdx.x] = threadIdx.x < a.k ? a.w[threadIdx.x] : 1.0f;
-    }
-    __syncthreads();
-    int u = blockIdx.x * kSingleWarps + warp;
-    int j = u % S, rp = u / S;  // slot and row pair of unit u
+    const int e = j < a.k ? a.idx[j] : a.E;
+    const float wj = j < a.k ? a.w[j] : 1.0f;
+    int rp = (int)(blockIdx.x / S) * kSingleWarps + warp;  // first row pair of this warp
     DownRegs X;
-    if (u < units) down_load(a, s_e[j], 2 * rp, lane, X);
-    stage_vectors<false>(a.h, a.F, S, [](int t) { return t; }, g, hs, corr);
+    if (rp < pairs) down_load(a, e, 2 * rp, lane, X);
+    stage_vectors<false>(a.h, a.F, 1, [j](int) { return j; }, g, hs, corr);
     __syncthreads();
 
-    const int dj = W % S, drp = W / S;  // unit stride W as (slot, row pair) steps
-    for (; u < units; u += W) {
+    for (; rp < pairs; rp += Wj) {
         float o0 = 0.f, o1 = 0.f;
-        down_compute(hs + (size_t)j * g.f4, corr + j * g.nch + lane, off, s_w[j], X, o0, o1);
-        const int jc = j, nc = 2 * rp;
-        j += dj;
-        rp += drp;
-        if (j >= S) {
-            j -= S;
-            ++rp;
-        }
-        if (u + W < units) down_load(a, s_e[j], 2 * rp, lane, X);
+        down_compute(hs, corr + lane, off, wj, X, o0, o1);
+        const int nc0 = 2 * rp;
+        if (rp + Wj < pairs) down_load(a, e, 2 * (rp + Wj), lane, X);
         o0 = warp_sum(o0);
         o1 = warp_sum(o1);
         if (lane == 0) {
-            a.partial[(size_t)jc * a.H + nc] = o0;
-            a.partial[(size_t)jc * a.H + nc + 1] = o1;
+            a.partial[(size_t)j * a.H + nc0] = o0;
+            a.partial[(size_t)j * a.H + nc0 + 1] = o1;
         }
     }
     griddep_launch_dependents();
