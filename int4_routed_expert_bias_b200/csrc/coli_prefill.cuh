@@ -12,7 +12,7 @@
 // Persistent CTAs (one per SM) walk the items; inside a CTA, warp roles:
 //   warp 0     TMA producer: int4 bytes + scales of the weight tile, 256 K at a
 //              time (3-deep ring), and the token rows (bf16), 64 K at a time
-//              (5-deep ring), straight into the 128-byte-swizzled layouts;
+//              (6-deep ring), straight into the 128-byte-swizzled layouts;
 //   warps 6..  dequantise: each thread owns one weight row (= TMEM lane) and
 //              a part of a 64-K step; q * s is formed in bf16 and written into a
 //              4-deep ring of A operands in TMEM with tcgen05.st;
@@ -44,7 +44,7 @@ constexpr int kPfMaxN = 192;      // tokens per tile (union group size on this p
 constexpr int kPfKStep = 64;      // K per MMA stage = one scale group
 constexpr int kPfRawK = 256;      // K per int4 stage
 constexpr int kPfRawStages = 3;
-constexpr int kPfBStages = 5;
+constexpr int kPfBStages = 6;
 constexpr int kPfAStages = 4;     // dequantised weight stages in TMEM, 32 columns each
 constexpr int kPfTmemCols = 512;
 constexpr int kPfACol = 2 * kPfMaxN;  // columns [0, 2 N_max): two accumulators; then the A ring
