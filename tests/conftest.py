@@ -10,6 +10,11 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # The layer library is built in-tree and not committed: build it once if a
+    # fresh checkout does not have it yet (nvcc cross-compiles without a GPU).
+    if not os.path.exists(os.path.join(ROOT, "int4_routed_expert_bias_b200", "libcoli.so")):
+        import __graft_entry__
+        __graft_entry__.build()
 
 
 def cuda_available():
