@@ -245,8 +245,8 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem,
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// cuTensorMapEncodeTiled from the driver, looked up once (the library links
-// only the runtime).  nullptr when the driver does not provide it.
+// cuTensorMapEncodeTiled from the CUDA driver, looked up once (the library links
+// only the runtime).  nullptr when the CUDA driver does not provide it.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
