@@ -401,9 +401,13 @@ def run_ours(args):
                     "bound": "hbm", "achieved": gu_gbs, "peak": hbm_peak, "unit": "GB/s",
                     "frac": gu_gbs / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
                     "alg_bytes_per_launch": gu_alg}
+    expert_alg = float(np.mean((U + 1) * c.expert_bytes))  # selected experts' int4 + scales only
     extra = {"graph_calls": G, "parallelism": f"replicas x{world}", "mean_union_U": float(U.mean()),
              "layer_alg_bytes_per_call": layer_alg, "layer_gbs": layer_gbs,
-             "layer_frac_of_hbm_peak": layer_gbs / hbm_peak, "stage_ms": stage_ms}
+             "layer_frac_of_hbm_peak": layer_gbs / hbm_peak,
+             "expert_alg_bytes_per_call": expert_alg,
+             "expert_frac_of_hbm_peak": expert_alg / (ms_per_step * 1e-3) / 1e9 / hbm_peak,
+             "stage_ms": stage_ms}
     if prefill:
         layer_flops = 2.0 * (c.T * c.k + c.T) * 3 * c.F * c.H + 2.0 * c.T * c.E * c.H
         extra["layer_tflops"] = layer_flops / (ms_per_step * 1e-3) / 1e12
