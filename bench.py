@@ -343,14 +343,23 @@ def run_ours(args):
         for i in range(G):
             coli.moe_profile_next(ev[i])
             call(i, with_idx=True)
+    # exactly K timed steps: K // G whole graphs, then one graph of the remaining K mod G calls
+    n_full, n_rem = divmod(max(1, args.steps), G)
+    g_rem = None
+    if n_rem:
+        g_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_rem, stream=cap):
+            for i in range(n_rem):
+                call(i)
     coli.moe_profile_next(None)
     torch.cuda.synchronize()
     g_plain.replay()
-    g_prof.replay()
+    g_prof.replay()  # fills the stage events and routing also when K < G (no profiled replay is timed)
+    if g_rem is not None:
+        g_rem.replay()
     torch.cuda.synchronize()
 
-    n_graphs = max(1, args.steps // G)
-    steps = n_graphs * G
+    steps = n_full * G + n_rem
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
@@ -360,9 +369,12 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     s = torch.cuda.current_stream()
     t0.record(s)
-    for _ in range(n_graphs - 1):
+    for _ in range(n_full - 1):
         g_plain.replay()
-    g_prof.replay()
+    if n_full >= 1:
+        g_prof.replay()  # the last whole graph carries the per-stage events
+    if g_rem is not None:
+        g_rem.replay()
     t1.record(s)
     torch.cuda.synchronize()
     barrier(world)
