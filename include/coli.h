@@ -116,6 +116,18 @@ COLI_API coli_status coli_expert_union(const int32_t* topk_idx, int T, int k, in
  * (0 if the layer description is invalid). */
 COLI_API size_t coli_moe_workspace_size(const coli_moe_layer* layer, int T);
 
+/* Device status of a coli_moe_forward call (no counterpart on the pages: it
+ * reports on this library's own kernels).  Kernels whose warps wait on one
+ * another inside a launch bound every wait in time; a wait that runs out (a
+ * fault or stall elsewhere on the GPU) leaves the outputs undefined and sets a
+ * 32-bit status word in the workspace, which is 0 after a normal call.  This
+ * returns the byte offset of that word inside the workspace of a call with T
+ * tokens of this layer: read the 4 bytes after the call has completed (e.g. with
+ * cudaMemcpy).  Returns SIZE_MAX if the sizes are invalid, if T == 0, or if a
+ * call of this shape does not write the word (the one-token kernels have no such
+ * waits).  Host arithmetic only: launches nothing, touches no device memory. */
+COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
+
 /*
  * The whole layer: Route, Union, the expert FFNs and the weighted combine.
  *   out_t = sum_j topk_w[t,j] * FFN_{topk_idx[t,j]}(x_t) + FFN_shared(x_t)

@@ -30,6 +30,8 @@ _lib.coli_expert_union.restype = _i
 _lib.coli_expert_union.argtypes = [_p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
 _lib.coli_moe_workspace_size.restype = ctypes.c_size_t
 _lib.coli_moe_workspace_size.argtypes = [_p, _i]
+_lib.coli_moe_status_word_offset.restype = ctypes.c_size_t
+_lib.coli_moe_status_word_offset.argtypes = [_p, _i]
 _lib.coli_moe_forward.restype = _i
 _lib.coli_moe_forward.argtypes = [_p, _p, _i, _i, _p, _i, _p, ctypes.c_size_t, _p, _p, _p]
 _lib.coli_moe_forward_noalloc.restype = _i
@@ -127,6 +129,13 @@ def expert_union(topk_idx, E, count, offset, active, n_active, perm, inv_perm, s
 
 def moe_workspace_size(layer, T):
     return int(_lib.coli_moe_workspace_size(layer.ref, T))
+
+
+def moe_status_word_offset(layer, T):
+    """Byte offset of the device status word in the workspace of a call with T
+    tokens, or None when such a call does not write it."""
+    off = int(_lib.coli_moe_status_word_offset(layer.ref, T))
+    return None if off == ctypes.c_size_t(-1).value else off
 
 
 def moe_forward(layer, x, out, workspace, topk_idx_out=None, topk_w_out=None, stream=None, T=None):

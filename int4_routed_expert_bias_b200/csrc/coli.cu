@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdint>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -361,6 +362,16 @@ size_t coli_moe_workspace_size(const coli_moe_layer* L, int T)
 {
     if (check_layer(L, T) != COLI_OK) return 0;
     return layout(nullptr, T, L->hidden, L->ffn, L->n_experts, L->top_k).bytes;
+}
+
+size_t coli_moe_status_word_offset(const coli_moe_layer* L, int T)
+{
+    if (check_layer(L, T) != COLI_OK || T == 0) return SIZE_MAX;
+    // the one-token chain (see coli_moe_forward) runs no union kernel, which is what zeroes the word
+    if (T == 1 && L->n_experts <= 256 && L->hidden == 1024 * 2 * kHalf && L->ffn == 2048) return SIZE_MAX;
+    char* const base = reinterpret_cast<char*>(256);  // any aligned base: only differences are used
+    const Workspace w = layout(base, T, L->hidden, L->ffn, L->n_experts, L->top_k);
+    return (size_t)(reinterpret_cast<char*>(w.ctl + 3) - base);
 }
 
 coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype xt, int T, void* out,

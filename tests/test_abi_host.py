@@ -73,6 +73,31 @@ def test_workspace_size_is_positive_and_grows(coli):
     assert coli.lib().coli_moe_workspace_size(ctypes.byref(_layer(coli, hidden=100)), 1) == 0
 
 
+def test_status_word_offset(coli):
+    """The device status word sits inside the workspace of the call it belongs
+    to, 4-byte aligned; calls that do not write it (one-token chain, empty
+    batches, invalid layers) report none."""
+    none = ctypes.c_size_t(-1).value
+    lib = coli.lib()
+    s = _layer(coli)
+    for T in (2, 4, 64, 65, 4096):
+        off = lib.coli_moe_status_word_offset(ctypes.byref(s), T)
+        assert off != none and off % 4 == 0
+        assert off + 4 <= lib.coli_moe_workspace_size(ctypes.byref(s), T)
+    assert lib.coli_moe_status_word_offset(ctypes.byref(s), 1) == none  # one-token chain
+    assert lib.coli_moe_status_word_offset(ctypes.byref(s), 0) == none
+    assert lib.coli_moe_status_word_offset(None, 4) == none
+    assert lib.coli_moe_status_word_offset(ctypes.byref(_layer(coli, hidden=100)), 4) == none
+    # one token of another shape goes through the union, which writes the word
+    small = _layer(coli, hidden=1024, ffn=512, n_experts=64)
+    assert lib.coli_moe_status_word_offset(ctypes.byref(small), 1) != none
+    # the Python binding maps "none" to None
+    L = coli.Layer.__new__(coli.Layer)
+    L.struct = s
+    assert coli.moe_status_word_offset(L, 1) is None
+    assert coli.moe_status_word_offset(L, 4) == lib.coli_moe_status_word_offset(ctypes.byref(s), 4)
+
+
 @pytest.mark.parametrize("over,status", [
     (dict(hidden=100), 1), (dict(hidden=0), 1), (dict(ffn=96), 1), (dict(top_k=0), 1),
     (dict(top_k=33), 1), (dict(n_experts=4, top_k=8), 1), (dict(n_experts=2000), 1),

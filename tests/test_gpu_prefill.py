@@ -67,6 +67,8 @@ def test_prefill_matches_oracle(env, H, F, E, k, T, xdt, odt):
     w = torch.empty((T, k), dtype=torch.float32, device="cuda")
     coli.moe_forward(L, xd, out, ws, idx, w)
     torch.cuda.synchronize()
+    off = coli.moe_status_word_offset(L, T)  # device status of the call: 0 unless a bounded wait ran out
+    assert off is not None and int(ws[off:off + 4].view(torch.int32).item()) == 0
     ridx, rw, rout = oracle.moe_layer(x, H, F, E, k, c.routed_scale, w_router, sel_bias, ex)
     assert np.array_equal(idx.cpu().numpy(), ridx)
     np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6)
