@@ -135,12 +135,16 @@ COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
  * The pages name the routed experts, the shared expert ("Colibri 完全ガイド",
  * DeepSeek-V3 router row) and int4 weights with one scale per 64; the SwiGLU
  * form of the expert and the unscaled, always-on shared expert are this
- * library's reading of them.  Activations and accumulation are fp32 (bf16 x is
- * widened exactly); out is written as fp32 or bf16 (round to nearest even).
+ * library's reading of them.  The router is fp32.  Batches of up to 64 tokens
+ * compute the experts in fp32 (bf16 x is widened exactly); larger batches run
+ * them on the tensor cores with bf16 operands (weights q * scale, activations
+ * and the SwiGLU output rounded to bf16) and fp32 accumulation.  out is written
+ * as fp32 or bf16 (round to nearest even).
  * x [T, H] dtype xt; out [T, H] dtype ot; workspace of at least
- * coli_moe_workspace_size(layer, T) bytes, contents undefined on entry and
- * exit, not shared by calls that may run concurrently.  topk_idx_out [T, k]
- * and topk_w_out [T, k] are optional copies of the routing (NULL to skip).
+ * coli_moe_workspace_size(layer, T) bytes, contents undefined on entry and on
+ * exit apart from the status word (coli_moe_status_word_offset), not shared by
+ * calls that may run concurrently.  topk_idx_out [T, k] and topk_w_out [T, k]
+ * are optional copies of the routing (NULL to skip).
  */
 COLI_API coli_status coli_moe_forward(const coli_moe_layer* layer, const void* x, coli_dtype xt, int T,
                              void* out, coli_dtype ot, void* workspace, size_t ws_bytes,
