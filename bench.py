@@ -6,14 +6,18 @@ A step is one layer call (Route, Union, gate/up + SwiGLU, down, combine) on one
 batch of synthetic activations.  Eight HBM-resident layers (expert weights
 generated on the device, 5.46 GB each at the full shape) are cycled, so the
 selected experts of a call (191 MB at batch 1) never sit in L2 from the call
-before.  The default workload is decode batch 1 (config 1).  Steps are
-captured in CUDA graphs of G calls; the timed region replays them, bracketed by
-a barrier and a device synchronise, timed with CUDA events; multi-GPU runs are
-independent replicas (no collective on the data path) and report the max over
-ranks.
+before.  Without --config the run measures the four workloads of the metric,
+batch 1, 4, 64 and 4096: the JSON line's value is batch 1 (the headline) and
+config.per_workload carries the other three.  Steps are captured in CUDA graphs
+of G calls; the timed region (exactly K steps, bracketed by a barrier and a
+device synchronise, timed with CUDA events) is replayed several times and the
+median is reported with its p10/p90.  Multi-GPU runs are independent replicas
+(no collective on the data path) and report the max over ranks.
 """
 import argparse
+import datetime
 import json
+import math
 import os
 import subprocess
 import sys
@@ -31,34 +35,41 @@ METRIC = "MoE-layer tokens/s and achieved HBM GB/s (% roofline) at batch 1/4/64/
 SEED = 1234
 N_LAYERS = 8  # resident layers cycled (bench --layers overrides it for profiling runs)
 STAGE_NAMES = ("route", "union", "gateup", "down", "combine")
+WORKLOADS = (1, 2, 3, 4)
+# nominal ms per step, only to size the number of timed replays (the same on every rank)
+NOMINAL_MS = {1: 0.06, 2: 0.3, 3: 3.0, 4: 5.0}
+TIMED_TARGET_S = 0.3  # aim for about this much timed work per workload
 
 
-def kernels_per_call(T, E):
-    """Our kernel launches in one layer call: batch 1 runs router scores, top-k,
-    gate/up, down and combine; decode batches run router scores, top-k +
-    union (one kernel up to 256 tokens), gate/up, down and combine; prefill
-    batches add the token-row gather in front of the two grouped GEMMs."""
-    if T == 1:
-        return 5
+def kernels_per_call(path, T, E):
+    """Our kernel launches in one layer call, by kernel chain: the one-token
+    chain runs router scores, top-k, gate/up, down and combine; the CUDA-core
+    decode chain runs router scores, top-k + union (one kernel up to 256
+    tokens), gate/up, down and combine; the prefill chain runs router scores,
+    (top-k,) union, the token-row gather, two grouped GEMMs and the slot sum."""
     fused = T <= 256 and E <= 256
-    if T <= 64:
+    if path == "single":
+        return 5
+    if path == "decode":
         return 5 if fused else 6
     return 6 if fused else 7
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20480)
-    ap.add_argument("--warmup", type=int, default=16)
-    ap.add_argument("--config", type=int, default=1, choices=[1, 2, 3, 4])
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--config", type=int, default=0, choices=[0, 1, 2, 3, 4],
+                    help="one workload only (0 = all four, batch 1 as the headline)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=8, help="resident layers cycled (profiling: fewer)")
     ap.add_argument("--experts", type=int, default=0,
                     help="routed experts per layer (0 = the workload's; profiling: fewer, same per-call bytes)")
+    ap.add_argument("--replays", type=int, default=0, help="timed replays of the K steps (0 = sized to ~0.3 s)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def measured_peaks():
@@ -80,15 +91,17 @@ def config_block(c, G, extra=None):
     d = {"workload": workload_desc(c), "cfg": c.cfg, "tokens_per_call": c.T, "hidden": c.H, "ffn": c.F,
          "experts": c.E, "top_k": c.k, "layers": N_LAYERS, "x_dtype": c.x_dtype, "out_dtype": c.out_dtype,
          "activation_pool": f"{G} distinct (step, layer) activation batches, replayed",
-         "l2": "inputs larger than L2: 8 layers x 5.46 GB cycled; a batch-1 call selects 191 MB"}
+         "l2": "inputs larger than L2: 8 layers x 5.46 GB cycled, each call selects its own experts "
+               "(191 MB at batch 1); no flush between replays"}
     if extra:
         d.update(extra)
     return d
 
 
 class ClockSampler:
-    """nvidia-smi clock and throttle-reason samples during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock and throttle-reason samples; only those taken inside the
+    timed windows (host wall-clock intervals passed to stop()) are kept."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -100,40 +113,49 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+        time.sleep(0.4)  # nvidia-smi's own start-up; the timed region begins after it
 
-    def stop(self):
+    @staticmethod
+    def _parse_time(s):
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(s, fmt)
+            except ValueError:
+                pass
+        return None
+
+    def stop(self, windows):
         if self.proc is None:
             return None
-        time.sleep(0.15)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
-        sm, mx, reasons = [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for r in rows:
-            r = [v.strip() for v in r]
-            if len(r) < 9:
+        rows = []
+        for r in out.strip().splitlines():
+            r = [v.strip() for v in r.split(",")]
+            if len(r) < 10:
                 continue
+            t = self._parse_time(r[0])
             try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
+                rows.append((t, float(r[2]), float(r[3]), r[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, r[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        inside = [x for x in rows if x[0] is not None and any(a <= x[0] <= b for a, b in windows)]
+        use = inside if inside else rows
+        reasons = sorted({n for x in use for n, v in zip(names, x[3]) if v.lower() == "active"})
+        sm = [x[1] for x in use]
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(x[2] for x in use)),
+                "samples": len(use), "samples_inside_timed_region": len(inside), "reasons": reasons}
 
 
 # ---------------------------------------------------------------------------
@@ -147,14 +169,15 @@ def dist_env():
 
 
 def max_over_ranks(value, world, torch):
-    """The largest `value` over all ranks (every rank gets it)."""
+    """The largest `value` (a number or a list of numbers, element-wise) over all ranks."""
     if world == 1:
         return value
     import torch.distributed as dist
     dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
-    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    t = torch.tensor(value if isinstance(value, list) else [value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    v = t.cpu().tolist()
+    return v if isinstance(value, list) else float(v[0])
 
 
 def job_throughput(world, steps, tokens_per_step, ms_max):
@@ -182,7 +205,7 @@ def time_oracle_calls(c, xs, routers, get_expert, budget_s, max_calls):
     import oracle
     done, spent = 0, 0.0
     for i in range(max_calls):
-        layer = i % N_LAYERS
+        layer = i % len(routers)
         x = xs[i % len(xs)]
         w_router, sel_bias = routers[layer]
         idx, _ = oracle.route(x, w_router, sel_bias, c.k, c.routed_scale)
@@ -197,16 +220,21 @@ def time_oracle_calls(c, xs, routers, get_expert, budget_s, max_calls):
     return done, spent, oracle.threads()
 
 
+def sample_config(c):
+    """The oracle's bounded sample of a workload: prefill calls are timed on 8 of
+    their tokens (tokens are independent; one full call is ~1.4e12 f64
+    multiply-adds)."""
+    if c.T > 64:
+        return inputs.Config(c.cfg, c.name, c.H, c.F, c.E, c.k, 8, c.x_dtype, c.out_dtype, c.layers)
+    return c
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    c = inputs.CONFIGS[args.config]
-    if c.T > 64:
-        # one prefill call is ~1.4e12 f64 multiply-adds; the sample is a token subset
-        c_sample = inputs.Config(c.cfg, c.name, c.H, c.F, c.E, c.k, 8, c.x_dtype, c.out_dtype, c.layers)
-    else:
-        c_sample = c
+    c = inputs.CONFIGS[args.config or 1]
+    c_sample = sample_config(c)
     routers = [inputs.router_params(c, SEED, l) for l in range(N_LAYERS)]
     xs = [inputs.activations(c_sample, SEED, s, s % N_LAYERS) for s in range(16)]
     cache = {}
@@ -270,39 +298,41 @@ def traffic_from_profiles(kernel, workload):
         return None
 
 
-def run_ours(args):
-    import torch
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    import int4_routed_expert_bias_b200 as coli
+# the dominant kernel of each kernel chain, the stage whose events bracket it,
+# and the name of its committed ncu summary
+DOMINANT = {
+    "single": ("gateup_single_kernel", "gateup", "gateup"),
+    "decode": ("expert_phase_kernel<gateup>", "gateup", "gateup-phase"),
+    "prefill": ("prefill_gemm_kernel<gate/up>", "gateup", "prefill-gemm"),
+}
 
-    global N_LAYERS
-    N_LAYERS = args.layers
-    c = inputs.CONFIGS[args.config]
-    if args.experts:
-        c = inputs.Config(c.cfg, f"{c.name}-E{args.experts}", c.H, c.F, args.experts, c.k, c.T, c.x_dtype,
-                          c.out_dtype, args.layers)
-    seed = SEED + 1000 * rank
-    hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
 
-    # eight resident layers, expert weights generated on the device
-    layers, bufs, routers = [], [], []
+def percentile(v, q):
+    return float(np.percentile(np.asarray(v, np.float64), q))
+
+
+class Resident:
+    """Eight resident layers of expert weights (shared by the full-shape workloads)."""
+
+    def __init__(self, torch, c, seed, n_layers):
+        self.bufs = [inputs.device_layer_tensors(torch, c, seed, l) for l in range(n_layers)]
+        self.H, self.F, self.E = c.H, c.F, c.E
+
+
+def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sampler_index):
+    """Time one workload; returns the fields of its benchmark entry."""
+    hbm_peak, bf16_peak, bf16_sust, peak_kind = peaks
+    routers, layers = [], []
     for l in range(N_LAYERS):
-        b = inputs.device_layer_tensors(torch, c, seed, l)
         w_router, sel_bias = inputs.router_params(c, seed, l)
         routers.append((w_router, sel_bias))
+        b = res.bufs[l]
         layers.append(coli.Layer(c.H, c.F, c.E, c.k, c.routed_scale, torch.from_numpy(w_router).cuda(),
                                  torch.from_numpy(sel_bias).cuda(), b["gate_q"], b["gate_s"], b["up_q"],
                                  b["up_s"], b["down_q"], b["down_s"]))
-        bufs.append(b)
-    torch.cuda.synchronize()
+    path = coli.moe_path(layers[0], c.T)
 
-    # activation pool: G distinct (step, layer) batches, G a multiple of 8
+    # activation pool: G distinct (step, layer) batches, G a multiple of the layer count
     reps = max(1, min(32, 4_000_000 // (c.T * c.H)))
     G = N_LAYERS * reps
     xs_host = [inputs.activations(c, seed, s // N_LAYERS, s % N_LAYERS) for s in range(G)]
@@ -323,7 +353,8 @@ def run_ours(args):
                          idx_dev[i % G] if with_idx else None, None)
 
     # warm-up (also the library's one-time per-device set-up), outside any graph
-    for i in range(max(args.warmup, 3)):
+    warm = max(args.warmup, 3)
+    for i in range(warm):
         call(i)
     torch.cuda.synchronize()
 
@@ -360,83 +391,94 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     steps = n_full * G + n_rem
-    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if args.replays:
+        R = args.replays
+    else:
+        R = int(min(100, max(5, math.ceil(TIMED_TARGET_S * 1e3 / (steps * NOMINAL_MS[c.cfg])))))
+    s = torch.cuda.current_stream()
+
+    def timed_region(last):
+        for _ in range(n_full - 1):
+            g_plain.replay()
+        if n_full >= 1:
+            (g_prof if last else g_plain).replay()  # the last replay's last whole graph carries the stage events
+        if g_rem is not None:
+            g_rem.replay()
+
+    sampler = ClockSampler(sampler_index) if rank == 0 else None
     if sampler:
         sampler.start()
+    ms_list, windows = [], []
+    for r in range(R):
+        barrier(world)
+        torch.cuda.synchronize()
+        w0 = datetime.datetime.now()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(s)
+        timed_region(r == R - 1)
+        t1.record(s)
+        torch.cuda.synchronize()
+        windows.append((w0, datetime.datetime.now()))
+        ms_list.append(t0.elapsed_time(t1))
     barrier(world)
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    s = torch.cuda.current_stream()
-    t0.record(s)
-    for _ in range(n_full - 1):
-        g_plain.replay()
-    if n_full >= 1:
-        g_prof.replay()  # the last whole graph carries the per-stage events
-    if g_rem is not None:
-        g_rem.replay()
-    t1.record(s)
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks = sampler.stop() if sampler else None
-    ms = t0.elapsed_time(t1)
-    ms_max = max_over_ranks(ms, world, torch)
-    ms_per_step = ms_max / steps
-    value = job_throughput(world, steps, c.T, ms_max)
+    clocks = sampler.stop(windows) if sampler else None
+    ms_max = max_over_ranks(ms_list, world, torch)
+    ms_med = float(np.median(ms_max))
+    ms_per_step = ms_med / steps
+    value = job_throughput(world, steps, c.T, ms_med)
 
-    # stage timings of the last G calls (inside the timed region)
+    # stage timings of the last G calls (inside the last timed replay)
     stage_ms = {n: float(np.mean([ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]) for i in range(G)]))
                 for j, n in enumerate(STAGE_NAMES)}
     idx_all = idx_dev.cpu().numpy()
     U = np.array([len(np.unique(idx_all[i])) for i in range(G)], np.float64)
     gu_bytes_per_expert = 2 * (c.F * c.H // 2 + c.F * c.H // 64 * 4)
     x_bytes = c.T * c.H * (2 if c.x_dtype == "bf16" else 4)
-    gu_alg = float(np.mean((U + 1) * gu_bytes_per_expert)) + x_bytes
-    gu_gbs = gu_alg / (stage_ms["gateup"] * 1e-3) / 1e9
-    layer_alg = float(np.mean((U + 1) * c.expert_bytes)) + c.E * c.H * 4 + c.E * 4 + x_bytes \
-        + c.T * c.H * (2 if c.out_dtype == "bf16" else 4)
+    out_bytes = c.T * c.H * (2 if c.out_dtype == "bf16" else 4)
+    layer_alg = float(np.mean((U + 1) * c.expert_bytes)) + c.E * c.H * 4 + c.E * 4 + x_bytes + out_bytes
     layer_gbs = layer_alg / (ms_per_step * 1e-3) / 1e9
-    traffic = traffic_from_profiles("gateup", c.name) if c.T <= 64 else traffic_from_profiles("gateup-gemm", c.name)
-
-    prefill = c.T > 64
+    kname, kstage, kfile = DOMINANT[path]
+    traffic = traffic_from_profiles(kfile, c.name)
+    prefill = path == "prefill"
     if prefill:
         # dominant kernel: the gate/up grouped GEMM, 2 * (pairs + shared) * 2F * H flops
         gu_flops = 2.0 * (c.T * c.k + c.T) * (2 * c.F) * c.H
-        gu_tflops = gu_flops / (stage_ms["gateup"] * 1e-3) / 1e12
-        roofline = {"kernel": "prefill_gemm_kernel<gate/up> (tcgen05 int4-dequant grouped GEMM + SwiGLU)",
+        gu_tflops = gu_flops / (stage_ms[kstage] * 1e-3) / 1e12
+        roofline = {"kernel": kname + " (tcgen05 int4-dequant grouped GEMM + SwiGLU)",
                     "bound": "tensor", "achieved": gu_tflops, "peak": bf16_sust, "unit": "TFLOP/s",
-                    "frac": gu_tflops / bf16_sust, "traffic": traffic, "peak_kind": peak_kind + " (sustained bf16)",
-                    "alg_flops_per_launch": gu_flops}
+                    "frac": gu_tflops / bf16_sust, "traffic": traffic,
+                    "peak_kind": peak_kind + " (sustained bf16)", "alg_flops_per_launch": gu_flops,
+                    "launch_ms": stage_ms[kstage]}
     else:
-        roofline = {"kernel": ("gateup_single_kernel" if c.T == 1 else "expert_phase_kernel<gateup>")
-                    + " (gate/up + SwiGLU, routed and shared experts)",
+        gu_alg = float(np.mean((U + 1) * gu_bytes_per_expert)) + x_bytes
+        gu_gbs = gu_alg / (stage_ms[kstage] * 1e-3) / 1e9
+        roofline = {"kernel": kname + " (gate/up + SwiGLU, routed and shared experts)",
                     "bound": "hbm", "achieved": gu_gbs, "peak": hbm_peak, "unit": "GB/s",
                     "frac": gu_gbs / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
-                    "alg_bytes_per_launch": gu_alg}
+                    "alg_bytes_per_launch": gu_alg, "launch_ms": stage_ms[kstage]}
+    if traffic is not None:
+        alg = roofline.get("alg_bytes_per_launch")
+        roofline["traffic_over_alg"] = traffic / alg if alg else None
     expert_alg = float(np.mean((U + 1) * c.expert_bytes))  # selected experts' int4 + scales only
-    extra = {"graph_calls": G, "parallelism": f"replicas x{world}", "mean_union_U": float(U.mean()),
+    entry = {"workload": workload_desc(c), "tokens_per_call": c.T, "path": path, "value": value,
+             "unit": "tokens/s", "steps": steps, "timed_replays": R, "ms_per_step": ms_per_step,
+             "ms_per_step_p10": percentile(ms_max, 10) / steps, "ms_per_step_p90": percentile(ms_max, 90) / steps,
+             "roofline": roofline, "gpu_launches": steps * kernels_per_call(path, c.T, c.E),
+             "mean_union_U": float(U.mean()), "max_union_U": float(U.max()),
              "layer_alg_bytes_per_call": layer_alg, "layer_gbs": layer_gbs,
              "layer_frac_of_hbm_peak": layer_gbs / hbm_peak,
              "expert_alg_bytes_per_call": expert_alg,
              "expert_frac_of_hbm_peak": expert_alg / (ms_per_step * 1e-3) / 1e9 / hbm_peak,
-             "stage_ms": stage_ms}
+             "stage_ms": stage_ms, "graph_calls": G, "clocks": clocks}
     if prefill:
         layer_flops = 2.0 * (c.T * c.k + c.T) * 3 * c.F * c.H + 2.0 * c.T * c.E * c.H
-        extra["layer_tflops"] = layer_flops / (ms_per_step * 1e-3) / 1e12
-        extra["layer_frac_of_bf16_sustained"] = extra["layer_tflops"] / bf16_sust
-
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if prefill else "f32", "data": "synthetic",
-            "config": config_block(c, G, extra),
-            "roofline": roofline,
-            "gpu_launches": steps * kernels_per_call(c.T, c.E),
-            "clocks": clocks}
+        entry["layer_tflops"] = layer_flops / (ms_per_step * 1e-3) / 1e12
+        entry["layer_frac_of_bf16_sustained"] = entry["layer_tflops"] / bf16_sust
 
     # end to end through the public call with host buffers: pinned x in, out back
     if not args.no_e2e:
-        n_e2e = min(steps, 2048)
+        n_e2e = 16 if prefill else min(max(steps, 64), 1024)
         xh = [torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).pin_memory() for x in xs_host]
         xin = torch.empty_like(xs[0])
         oh = torch.empty((c.T, c.H), dtype=odt).pin_memory()
@@ -453,9 +495,9 @@ def run_ours(args):
         e1.record(s)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world, torch)
-        line["e2e"] = {"value": job_throughput(world, n_e2e, c.T, ems), "unit": "tokens/s",
-                       "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
-                       "steps": n_e2e, "host_sync_per_step": True}
+        entry["e2e"] = {"value": job_throughput(world, n_e2e, c.T, ems), "unit": "tokens/s",
+                        "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+                        "steps": n_e2e, "host_sync_per_step": True}
 
     # the oracle on this machine's host cores, bounded sample, rank 0 at N=1 only
     if world == 1 and not args.no_cpu:
@@ -463,22 +505,78 @@ def run_ours(args):
 
         def get_expert(layer, e):
             if (layer, e) not in cache:
-                cache[(layer, e)] = expert_host_copy(bufs[layer], e)
+                cache[(layer, e)] = expert_host_copy(res.bufs[layer], e)
             return cache[(layer, e)]
 
-        c_sample = c if c.T <= 64 else inputs.Config(c.cfg, c.name, c.H, c.F, c.E, c.k, 8, c.x_dtype,
-                                                     c.out_dtype, c.layers)
+        c_sample = sample_config(c)
         xs_cpu = [x[: c_sample.T] for x in xs_host[:16]]
-        n, spent, cores = time_oracle_calls(c_sample, xs_cpu, routers, get_expert, 15.0, 64)
-        line["cpu_baseline"] = {"value": n * c_sample.T / spent, "unit": "tokens/s", "cores": cores,
-                                "kind": "oracle",
-                                "sample": f"{n} layer calls of {c_sample.T} token(s), about 15 s of oracle time"}
+        budget = 15.0 if c.cfg == 1 else 6.0
+        n, spent, cores = time_oracle_calls(c_sample, xs_cpu, routers, get_expert, budget, 64)
+        entry["cpu_baseline"] = {"value": n * c_sample.T / spent, "unit": "tokens/s", "cores": cores,
+                                 "kind": "oracle",
+                                 "sample": f"{n} layer calls of {c_sample.T} token(s), about {budget:.0f} s "
+                                           f"of oracle time"}
+    del g_plain, g_prof, g_rem
+    return entry
 
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import int4_routed_expert_bias_b200 as coli
+
+    global N_LAYERS
+    N_LAYERS = args.layers
+    cfgs = [args.config] if args.config else list(WORKLOADS)
+    seed = SEED + 1000 * rank
+    peaks = measured_peaks()
+
+    def cfg_of(k):
+        c = inputs.CONFIGS[k]
+        if args.experts:
+            c = inputs.Config(c.cfg, f"{c.name}-E{args.experts}", c.H, c.F, args.experts, c.k, c.T, c.x_dtype,
+                              c.out_dtype, args.layers)
+        return c
+
+    res = Resident(torch, cfg_of(cfgs[0]), seed, N_LAYERS)  # expert weights depend on (seed, layer) only
+    torch.cuda.synchronize()
+    entries = {}
+    for k in cfgs:
+        entries[k] = measure_workload(args, torch, coli, cfg_of(k), res, seed, world, rank, peaks,
+                                      torch.cuda.current_device())
+        torch.cuda.empty_cache()
+
+    head_cfg = cfgs[0]
+    head, c = entries[head_cfg], cfg_of(head_cfg)
+    extra = {"parallelism": f"replicas x{world}", "path": head["path"], "mean_union_U": head["mean_union_U"],
+             "timed_replays": head["timed_replays"], "ms_per_step_p10": head["ms_per_step_p10"],
+             "ms_per_step_p90": head["ms_per_step_p90"],
+             "layer_alg_bytes_per_call": head["layer_alg_bytes_per_call"], "layer_gbs": head["layer_gbs"],
+             "layer_frac_of_hbm_peak": head["layer_frac_of_hbm_peak"],
+             "expert_alg_bytes_per_call": head["expert_alg_bytes_per_call"],
+             "expert_frac_of_hbm_peak": head["expert_frac_of_hbm_peak"], "stage_ms": head["stage_ms"],
+             "timing": "median of the timed replays of exactly K steps (CUDA events, max over ranks)"}
+    if len(cfgs) > 1:
+        extra["per_workload"] = {cfg_of(k).name: entries[k] for k in cfgs[1:]}
+    line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": head["steps"],
+            "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if head["path"] == "prefill" else "f32", "data": "synthetic",
+            "config": config_block(c, head["graph_calls"], extra),
+            "roofline": head["roofline"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"]}
+    if "e2e" in head:
+        line["e2e"] = head["e2e"]
+    if "cpu_baseline" in head:
+        line["cpu_baseline"] = head["cpu_baseline"]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del g_plain, g_prof
         dist.destroy_process_group()
     return 0
 

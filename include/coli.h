@@ -150,6 +150,24 @@ COLI_API coli_status coli_moe_forward(const coli_moe_layer* layer, const void* x
                              void* out, coli_dtype ot, void* workspace, size_t ws_bytes,
                              int32_t* topk_idx_out, float* topk_w_out, cudaStream_t stream);
 
+/* Kernel chains of coli_moe_forward (coli_moe_path). */
+enum {
+    COLI_PATH_NONE = 0,     /* empty batch or invalid arguments: nothing runs */
+    COLI_PATH_SINGLE = 1,   /* one token at hidden 6144, ffn 2048, <= 256 experts: the one-token chain */
+    COLI_PATH_DECODE = 2,   /* CUDA-core int4 GEMV kernels (fp32 arithmetic) */
+    COLI_PATH_PREFILL = 3   /* tcgen05 tensor-core grouped GEMMs (bf16 operands, fp32 accumulation) */
+};
+
+/*
+ * Which kernel chain coli_moe_forward runs for a batch of T tokens of this
+ * layer.  Decided by the shapes alone: more than 64 tokens with hidden and ffn
+ * multiples of 256 take the tensor-core path (a device without
+ * cuTensorMapEncodeTiled in its driver then gets COLI_ERR_UNSUPPORTED from
+ * coli_moe_forward, never another path); every other valid batch runs on CUDA
+ * cores in fp32.  Host-only, launches nothing.
+ */
+COLI_API int coli_moe_path(const coli_moe_layer* layer, int T);
+
 /* Stages of coli_moe_forward, for coli_moe_profile_next(). */
 enum {
     COLI_STAGE_ROUTE = 0,   /* router scores and top-k */
@@ -193,7 +211,9 @@ COLI_API coli_status coli_moe_profile_next(cudaEvent_t* events, int n_events);
  *   - Every GPU that loads the library holds the 8 MiB array until the process
  *     exits.  The first call on each device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current; make that first
- *     call before any stream capture.
+ *     call before any stream capture.  The address is kept for the life of
+ *     the process: do not call this entry point on a device after
+ *     cudaDeviceReset() (the array may then sit elsewhere).
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents (nothing in it needs to start at zero: every call writes what it
  *     reads).  Calls whose work may overlap on the GPU (different streams, or

@@ -16,6 +16,7 @@ F32, BF16 = 0, 1
 STATUS = {0: "COLI_OK", 1: "COLI_ERR_INVALID_ARG", 2: "COLI_ERR_UNSUPPORTED", 3: "COLI_ERR_WORKSPACE",
           4: "COLI_ERR_CUDA"}
 STAGES = ("route", "union", "gateup", "down", "combine")
+PATHS = {0: "none", 1: "single", 2: "decode", 3: "prefill"}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
@@ -32,6 +33,8 @@ _lib.coli_moe_workspace_size.restype = ctypes.c_size_t
 _lib.coli_moe_workspace_size.argtypes = [_p, _i]
 _lib.coli_moe_status_word_offset.restype = ctypes.c_size_t
 _lib.coli_moe_status_word_offset.argtypes = [_p, _i]
+_lib.coli_moe_path.restype = _i
+_lib.coli_moe_path.argtypes = [_p, _i]
 _lib.coli_moe_forward.restype = _i
 _lib.coli_moe_forward.argtypes = [_p, _p, _i, _i, _p, _i, _p, ctypes.c_size_t, _p, _p, _p]
 _lib.coli_moe_forward_noalloc.restype = _i
@@ -129,6 +132,13 @@ def expert_union(topk_idx, E, count, offset, active, n_active, perm, inv_perm, s
 
 def moe_workspace_size(layer, T):
     return int(_lib.coli_moe_workspace_size(layer.ref, T))
+
+
+def moe_path(layer, T):
+    """Name of the kernel chain moe_forward runs for T tokens of this layer:
+    "single" (one-token chain), "decode" (CUDA cores), "prefill" (tensor cores)
+    or "none" (empty or invalid call)."""
+    return PATHS[int(_lib.coli_moe_path(layer.ref, T))]
 
 
 def moe_status_word_offset(layer, T):

@@ -202,6 +202,22 @@ coli_status check_layer(const coli_moe_layer* L, int T)
     return COLI_OK;
 }
 
+// Argument checks of a layer call other than its workspace (host only).
+coli_status check_call(const coli_moe_layer* L, const void* x, coli_dtype xt, int T, const void* out, coli_dtype ot,
+                       const int32_t* topk_idx_out, const float* topk_w_out)
+{
+    coli_status st = check_layer(L, T);
+    if (st != COLI_OK) return st;
+    if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown activation dtype %d", (int)xt);
+    if (ot != COLI_F32 && ot != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown output dtype %d", (int)ot);
+    if (T == 0) return COLI_OK;
+    if (!x || !out) return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(x, 16) || !aligned(out, 16)) return fail(COLI_ERR_INVALID_ARG, "x / out not 16-byte aligned");
+    if ((topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
+        return fail(COLI_ERR_INVALID_ARG, "routing outputs not 4-byte aligned");
+    return COLI_OK;
+}
+
 struct StageTimer {
     cudaEvent_t* ev = nullptr;
     int n = 0;
@@ -293,6 +309,17 @@ constexpr int kDecodeMaxT = 64;
 // Batches up to this size take the top-k inside the union block.
 constexpr int kFusedTopkMaxT = 256;
 
+// The kernel chain a valid call of T tokens runs (coli_moe_path), from the
+// shapes alone: every path's shared-memory needs fit the 227 KB per block of
+// sm_100, which the device set-up checks once.
+int choose_path(const coli_moe_layer* L, int T)
+{
+    if (T == 0) return COLI_PATH_NONE;
+    if (T == 1 && L->n_experts <= 256 && L->hidden == 1024 * 2 * kHalf && L->ffn == 2048) return COLI_PATH_SINGLE;
+    if (T > kDecodeMaxT && L->hidden % kPfRawK == 0 && L->ffn % kPfRawK == 0) return COLI_PATH_PREFILL;
+    return COLI_PATH_DECODE;
+}
+
 }  // namespace
 
 extern "C" {
@@ -364,11 +391,17 @@ size_t coli_moe_workspace_size(const coli_moe_layer* L, int T)
     return layout(nullptr, T, L->hidden, L->ffn, L->n_experts, L->top_k).bytes;
 }
 
+int coli_moe_path(const coli_moe_layer* L, int T)
+{
+    if (check_layer(L, T) != COLI_OK) return COLI_PATH_NONE;
+    return choose_path(L, T);
+}
+
 size_t coli_moe_status_word_offset(const coli_moe_layer* L, int T)
 {
     if (check_layer(L, T) != COLI_OK || T == 0) return SIZE_MAX;
-    // the one-token chain (see coli_moe_forward) runs no union kernel, which is what zeroes the word
-    if (T == 1 && L->n_experts <= 256 && L->hidden == 1024 * 2 * kHalf && L->ffn == 2048) return SIZE_MAX;
+    // the one-token chain runs no union kernel, which is what zeroes the word
+    if (choose_path(L, T) == COLI_PATH_SINGLE) return SIZE_MAX;
     char* const base = reinterpret_cast<char*>(256);  // any aligned base: only differences are used
     const Workspace w = layout(base, T, L->hidden, L->ffn, L->n_experts, L->top_k);
     return (size_t)(reinterpret_cast<char*>(w.ctl + 3) - base);
@@ -384,16 +417,10 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     g_prof_events = nullptr;  // one-shot
     g_prof_n = 0;
 
-    coli_status st = check_layer(L, T);
-    if (st != COLI_OK) return st;
-    if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown activation dtype %d", (int)xt);
-    if (ot != COLI_F32 && ot != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown output dtype %d", (int)ot);
-    if (T == 0) return COLI_OK;
-    if (!x || !out || !workspace) return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
-    if (!aligned(x, 16) || !aligned(out, 16)) return fail(COLI_ERR_INVALID_ARG, "x / out not 16-byte aligned");
+    coli_status st = check_call(L, x, xt, T, out, ot, topk_idx_out, topk_w_out);
+    if (st != COLI_OK || T == 0) return st;
+    if (!workspace) return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned(workspace, 256)) return fail(COLI_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-    if ((topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
-        return fail(COLI_ERR_INVALID_ARG, "routing outputs not 4-byte aligned");
     const int H = L->hidden, F = L->ffn, E = L->n_experts, k = L->top_k;
     Workspace w = layout(workspace, T, H, F, E, k);
     if (ws_bytes < w.bytes)
@@ -413,10 +440,10 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
 
     // One token: router scores, top-k, gate/up, down, combine; the union of a
     // one-token batch is its k experts.
+    const int path = choose_path(L, T);
     const size_t s1_gu = stage_smem_bytes(H, 1), s1_dn = stage_smem_bytes(F, 1);
     // (batch-1 path: see coli_decode1.cuh)
-    if (T == 1 && E <= 256 && H == 1024 * 2 * kHalf && F == 2048 &&
-        s1_gu <= (size_t)dev->smem_optin && s1_dn <= (size_t)dev->smem_optin) {
+    if (path == COLI_PATH_SINGLE) {
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
         st = launch_logits(x, xt, 1, H, L->w_router, E, w.logits, nullptr, 0, stream);
         if (st != COLI_OK) return st;
@@ -461,16 +488,21 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     const size_t Q = (size_t)T * k + T;
     uint16_t* xg = reinterpret_cast<uint16_t*>(w.partial);  // gathered rows; later reused for ys
     uint16_t* hb = reinterpret_cast<uint16_t*>(w.h);
-    const bool prefill = T > kDecodeMaxT && H % kPfRawK == 0 && F % kPfRawK == 0 &&
-                         (size_t)dev->smem_optin >= kPfSmemBytes &&
-                         encode_weight_maps(&m_gq, &m_gs, L->gate_q, L->gate_s, E, F, H) &&
+    if (path == COLI_PATH_PREFILL && (size_t)dev->smem_optin < kPfSmemBytes)
+        return fail(COLI_ERR_UNSUPPORTED, "the device offers %d bytes of shared memory per block; the prefill GEMM needs %zu",
+                    dev->smem_optin, kPfSmemBytes);
+    if (path == COLI_PATH_PREFILL && !tensor_map_encoder())
+        return fail(COLI_ERR_UNSUPPORTED, "the CUDA driver provides no cuTensorMapEncodeTiled (tensor-core prefill path)");
+    if (path == COLI_PATH_PREFILL &&
+        !(encode_weight_maps(&m_gq, &m_gs, L->gate_q, L->gate_s, E, F, H) &&
                          encode_weight_maps(&m_uq, &m_us, L->up_q, L->up_s, E, F, H) &&
                          encode_weight_maps(&m_dq, &m_ds, L->down_q, L->down_s, E, H, F) &&
                          encode_2d(&m_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xg, (uint64_t)H, Q, kPfKStep, kPfBRows,
                                    CU_TENSOR_MAP_SWIZZLE_128B) &&
                          encode_2d(&m_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, hb, (uint64_t)F, Q, kPfKStep, kPfBRows,
-                                   CU_TENSOR_MAP_SWIZZLE_128B);
-    if (prefill) {
+                                   CU_TENSOR_MAP_SWIZZLE_128B)))
+        return fail(COLI_ERR_CUDA, "cuTensorMapEncodeTiled rejected a prefill tensor map");
+    if (path == COLI_PATH_PREFILL) {
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
         {
             dim3 grid((T + kRtTile - 1) / kRtTile, (E + kRtTile - 1) / kRtTile);
@@ -626,11 +658,20 @@ extern "C" coli_status coli_moe_forward_noalloc(const coli_moe_layer* L, const v
                                                 void* out, coli_dtype ot, int32_t* topk_idx_out,
                                                 float* topk_w_out, cudaStream_t stream)
 {
-    const size_t need = coli_moe_workspace_size(L, T);  // 0 for an invalid layer: forward reports why
-    if (need > (size_t)COLI_NOALLOC_SCRATCH_BYTES)
+    // Every argument is checked before any CUDA call; a refused or empty call
+    // consumes an armed stage-timing hook, as coli_moe_forward would.
+    coli_status st0 = check_call(L, x, xt, T, out, ot, topk_idx_out, topk_w_out);
+    const size_t need = st0 == COLI_OK ? coli_moe_workspace_size(L, T) : 0;
+    if (st0 != COLI_OK || T == 0 || need > (size_t)COLI_NOALLOC_SCRATCH_BYTES) {
+        g_prof_events = nullptr;
+        g_prof_n = 0;
+    }
+    if (st0 != COLI_OK || T == 0) return st0;
+    if (need > (size_t)COLI_NOALLOC_SCRATCH_BYTES) {
         return fail(COLI_ERR_WORKSPACE,
                     "T=%d needs %zu bytes of scratch; the static scratch holds %zu bytes (use coli_moe_forward)",
                     T, need, (size_t)COLI_NOALLOC_SCRATCH_BYTES);
+    }
     void* ws = nullptr;
     coli_status st = noalloc_scratch(&ws);
     if (st != COLI_OK) return st;

@@ -9,8 +9,9 @@
 //   window A, bits 19..22:  fa = 1 + (q_a + 8) / 16
 //   window B, bits 15..18:  fb = 1 + (q_b + 8) / 256
 // (the nibble's top bit is flipped, so q + 8 = nibble ^ 8 for two's complement).
-// Shifts w<<15, w<<7 and, with t = w>>12, t<<11, t<<3 place nibbles (1,0),
-// (3,2), (5,4), (7,6) into (A,B); each float is one lop3.  A packed fp32x2 FMA then takes one odd-k and
+// The four shifts w<<15, w<<7, w>>1 and w>>9 place nibbles (1,0), (3,2), (5,4)
+// and (7,6) into (A,B); each float is one lop3, so a word costs 4 shifts and
+// 8 lop3 on the integer pipe.  A packed fp32x2 FMA then takes one odd-k and
 // one even-k product.  Over a chunk of 32 k values:
 //   sum_k q_k x_k = 16 * sum_odd fa x + 256 * sum_even fb x
 //                   - 24 * sum_odd x - 264 * sum_even x,
@@ -40,11 +41,10 @@ __device__ __forceinline__ float2 nib_pair(uint32_t s)
 // staged as swapped pairs: x01 = (x[8q+1], x[8q]), x23 = (x[8q+3], x[8q+2]), ...
 __device__ __forceinline__ float2 word_dot(uint32_t w, float4 xlo, float4 xhi, float2 acc)
 {
-    const uint32_t t = w >> 12;
     acc = __ffma2_rn(nib_pair(w << 15), make_float2(xlo.x, xlo.y), acc);
     acc = __ffma2_rn(nib_pair(w << 7), make_float2(xlo.z, xlo.w), acc);
-    acc = __ffma2_rn(nib_pair(t << 11), make_float2(xhi.x, xhi.y), acc);
-    acc = __ffma2_rn(nib_pair(t << 3), make_float2(xhi.z, xhi.w), acc);
+    acc = __ffma2_rn(nib_pair(w >> 1), make_float2(xhi.x, xhi.y), acc);
+    acc = __ffma2_rn(nib_pair(w >> 9), make_float2(xhi.z, xhi.w), acc);
     return acc;
 }
 

@@ -22,6 +22,30 @@ def rel_inf_err(y, ref):
     return float((num / den).max())
 
 
+def big_element_err(y, ref):
+    """Largest element-wise relative error over the elements that carry the
+    output: |r| > 0.1 * |r_t|_inf of their token (near-zero elements are
+    ill-conditioned for a relative measure)."""
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    big = np.abs(ref) > 0.1 * np.abs(ref).max(axis=-1, keepdims=True)
+    return float((np.abs(y - ref)[big] / np.abs(ref)[big]).max())
+
+
+def check_output(y, ref, tol, label=""):
+    """Assert the layer-output bound (per-token inf-norm relative error <= tol)
+    and the element-wise bound it implies on large elements (<= 10 tol); print
+    both with the largest absolute error.  Returns the inf-norm error."""
+    inf = rel_inf_err(y, ref)
+    elem = big_element_err(y, ref)
+    mabs = float(np.abs(np.asarray(y, np.float64) - ref).max())
+    print(f"{label}: inf-norm rel err {inf:.3e}, element rel err (|r| > 0.1 max) {elem:.3e}, "
+          f"max abs err {mabs:.3e} (tol {tol:g})")
+    assert inf <= tol, (label, inf)
+    assert elem <= 10 * tol, (label, elem)
+    return inf
+
+
 def near_ties(biased, k):
     """Tokens whose top-(k+1) biased scores have an adjacent gap below GAP."""
     top = -np.sort(-biased, axis=1)[:, : k + 1]

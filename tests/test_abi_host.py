@@ -32,7 +32,7 @@ def declared_functions():
 def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("coli_router_topk", "coli_expert_union", "coli_moe_workspace_size", "coli_moe_forward",
-              "coli_status_string", "coli_last_error", "coli_moe_profile_next"):
+              "coli_status_string", "coli_last_error", "coli_moe_profile_next", "coli_moe_path"):
         assert n in names
 
 
@@ -147,6 +147,22 @@ def test_union_rejects_bad_calls(coli):
     assert L.coli_expert_union(fake, 1, 8, 4, fake, fake, fake, fake, fake, fake, None) == 1
     assert L.coli_expert_union(fake, 1, 8, 256, None, fake, fake, fake, fake, fake, None) == 1
     assert L.coli_expert_union(None, 1, 8, 256, fake, fake, fake, fake, fake, fake, None) == 1
+
+
+def test_path_choice(coli):
+    """The kernel chain is chosen from the shapes alone, the same way the
+    forward call and the status-word query see it."""
+    L = coli.Layer.__new__(coli.Layer)
+    L.struct = _layer(coli)
+    assert [coli.moe_path(L, T) for T in (0, 1, 2, 64, 65, 4096)] == \
+        ["none", "single", "decode", "decode", "prefill", "prefill"]
+    L.struct = _layer(coli, hidden=256, ffn=128, n_experts=16, top_k=4)
+    assert coli.moe_path(L, 130) == "decode"  # ffn not a multiple of 256: CUDA cores at any batch
+    assert coli.moe_path(L, 1) == "decode"    # one token of another shape
+    L.struct = _layer(coli, hidden=256, ffn=256, n_experts=16, top_k=4)
+    assert coli.moe_path(L, 130) == "prefill"
+    L.struct = _layer(coli, hidden=100)
+    assert coli.moe_path(L, 4) == "none"
 
 
 def test_profile_hook_arms_and_disarms(coli):

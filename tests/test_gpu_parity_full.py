@@ -3,9 +3,13 @@ shared, top-8), through the same entry point and launch path the benchmark
 times, for the four full-size workloads (decode-1, verify-4, decode-64,
 prefill-4096).
 
-Routing and the union are compared for every token; the layer output for every
-token of the small batches and for sampled tokens of the large ones (the
-oracle computes tokens independently: a T-token call equals T one-token calls).
+Routing and the union are compared for every token.  The layer output is
+compared for every token of the decode batches (1, 4 and 64 tokens) and, for
+the 4096-token prefill, for tokens chosen so that every tile the tensor-core
+GEMMs compute is checked: one token from each 192-pair token tile of the shared
+expert, the first and last pair of 16 routed experts, and the first and last
+token (the oracle computes tokens independently: a T-token call equals T
+one-token calls).
 """
 import numpy as np
 import pytest
@@ -53,8 +57,25 @@ def test_device_generator_matches_host(full):
             assert np.array_equal(bufs[n][e].cpu().numpy(), h[n]), (e, n)
 
 
-@pytest.mark.parametrize("cfg,n_sample", [(1, 1), (2, 4), (3, 6), (4, 5)])
-def test_full_size_layer_matches_oracle(full, cfg, n_sample):
+PF_TILE = 192  # token-tile width of the prefill GEMMs (pairs of one expert per tile)
+
+
+def prefill_tokens(ridx, u, T, k, rng, n_experts=16):
+    """Tokens whose outputs cover every shared-expert token tile and both ends
+    of the token tiles of n_experts routed experts, plus tokens 0 and T-1."""
+    toks = {0, T - 1}
+    for b in range(0, T, PF_TILE):
+        toks.add(int(rng.integers(b, min(b + PF_TILE, T))))
+    active = u["active"][: u["n_active"]]
+    for e in rng.choice(active, size=min(n_experts, len(active)), replace=False):
+        first, last = u["offset"][e], u["offset"][e + 1] - 1
+        toks.add(int(u["perm"][first]) // k)
+        toks.add(int(u["perm"][last]) // k)
+    return np.array(sorted(toks))
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_full_size_layer_matches_oracle(full, cfg):
     coli, torch, bufs, host_expert = full
     c = inputs.CONFIGS[cfg]
     w_router, sel_bias = inputs.router_params(c, SEED, LAYER)
@@ -82,12 +103,13 @@ def test_full_size_layer_matches_oracle(full, cfg, n_sample):
     if cfg == 3:
         assert u["count"].max() > 8  # the Zipf bias makes hot experts
 
-    # outputs: sampled tokens against the oracle layer
+    # outputs: every token of a decode batch; the tile-covering sample of the prefill batch
+    assert coli.moe_path(L, T) == {1: "single", 2: "decode", 3: "decode", 4: "prefill"}[cfg]
     rng = np.random.default_rng(cfg)
-    tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, n_sample), replace=False)]))[:max(n_sample, 1)]
+    tokens = np.arange(T) if T <= 64 else prefill_tokens(ridx, u, T, c.k, rng)
+    assert tokens[-1] == T - 1
     need = set(ridx[tokens].ravel().tolist()) | {c.E}
     experts = {e: host_expert(e) for e in need}
     _, _, rout = oracle.moe_layer(x[tokens], c.H, c.F, c.E, c.k, c.routed_scale, w_router, sel_bias, experts)
-    tol = 1e-2 if c.out_dtype == "bf16" else S.TOL_DECODE
-    err = S.rel_inf_err(out[tokens], rout)
-    assert err <= tol, (cfg, err)
+    tol = S.TOL_PREFILL if T > 64 else S.TOL_DECODE
+    S.check_output(out[tokens], rout, tol, f"{c.name} ({len(tokens)} of {T} tokens)")

@@ -142,8 +142,36 @@ def test_ragged_batches(env, T):
     ridx, rw, rout = oracle.moe_layer(x, c.H, c.F, c.E, c.k, c.routed_scale, w_router, sel_bias, ex)
     assert np.array_equal(idx, ridx)
     np.testing.assert_allclose(w, rw, rtol=2e-6)
-    # batches above 64 tokens take the bf16 tensor-core prefill path
-    assert S.rel_inf_err(out, rout) <= (S.TOL_DECODE if T <= 64 else S.TOL_PREFILL)
+    # ffn 128 is not a multiple of 256: every batch, 130 tokens included, runs on CUDA cores in fp32
+    coli, torch = env
+    L = S.upload_layer(coli, torch, c, w_router, sel_bias, inputs.stack_experts(ex, c.E))
+    assert coli.moe_path(L, T) == "decode"
+    S.check_output(out, rout, S.TOL_DECODE, f"ragged T={T}")
+
+
+@pytest.mark.parametrize("T", [65, 130])
+def test_just_above_the_decode_batch_limit_takes_the_tensor_cores(env, T):
+    """65 and 130 tokens at hidden and ffn multiples of 256 run the tcgen05 prefill path."""
+    coli, torch = env
+    c = inputs.Config(0, "ragged-tc", 256, 256, 16, 4, T, "f32", "f32", 1)
+    rng = np.random.default_rng(300 + T)
+    ex = _random_experts(rng, c.H, c.F, c.E)
+    w_router = (rng.standard_normal((c.E, c.H)) * 0.05).astype(np.float32)
+    sel_bias = (rng.standard_normal(c.E) * 0.02).astype(np.float32)
+    x = rng.standard_normal((T, c.H)).astype(np.float32)
+    for _ in range(100):
+        _, _, (_, _, biased) = oracle.route(x, w_router, sel_bias, c.k, c.routed_scale, True)
+        bad = S.near_ties(biased, c.k)
+        if len(bad) == 0:
+            break
+        x[bad] = rng.standard_normal((len(bad), c.H)).astype(np.float32)
+    L = S.upload_layer(coli, torch, c, w_router, sel_bias, inputs.stack_experts(ex, c.E))
+    assert coli.moe_path(L, T) == "prefill"
+    idx, w, out = _run_layer(env, c, w_router, sel_bias, ex, x)
+    ridx, rw, rout = oracle.moe_layer(x, c.H, c.F, c.E, c.k, c.routed_scale, w_router, sel_bias, ex)
+    assert np.array_equal(idx, ridx)
+    np.testing.assert_allclose(w, rw, rtol=2e-6)
+    S.check_output(out, rout, S.TOL_PREFILL, f"tensor-core T={T}")
 
 
 def test_smallest_shapes_bf16_in_bf16_out(env):
