@@ -41,6 +41,11 @@ def lib():
         L.coli_oracle_moe_layer.restype = ctypes.c_int
         L.coli_oracle_moe_layer.argtypes = [_ptr, _i64, _i64, _i64, _i64, _i64, _dbl,
                                             _ptr, _ptr] + [_ptr] * 6 + [_ptr, _ptr, _ptr]
+        L.coli_oracle_route_top_p.restype = ctypes.c_int
+        L.coli_oracle_route_top_p.argtypes = [_ptr, _i64, _i64, _ptr, _ptr, _i64, _i64, _dbl, _dbl, _ptr, _ptr]
+        L.coli_oracle_moe_layer_top_p.restype = ctypes.c_int
+        L.coli_oracle_moe_layer_top_p.argtypes = [_ptr, _i64, _i64, _i64, _i64, _i64, _dbl, _dbl,
+                                                  _ptr, _ptr] + [_ptr] * 6 + [_ptr, _ptr, _ptr]
         L.coli_oracle_threads.restype = ctypes.c_int
         L.coli_oracle_threads.argtypes = []
         _lib = L
@@ -110,6 +115,20 @@ def route(x, w_router, sel_bias, k, routed_scale, want_scores=False):
     return idx, w
 
 
+def route_top_p(x, w_router, sel_bias, k, routed_scale, top_p):
+    """Top-k routing cut by adaptive expert top-p: (idx int32 [T,k], w f64 [T,k]);
+    dropped slots have index -1 and weight 0."""
+    x = _c(widen(x), np.float64)
+    T, H = x.shape
+    w_router = _c(w_router, np.float32); sel_bias = _c(sel_bias, np.float32)
+    E = w_router.shape[0]
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    _check(lib().coli_oracle_route_top_p(_p(x), T, H, _p(w_router), _p(sel_bias), E, k, float(routed_scale),
+                                         float(top_p), _p(idx), _p(w)), "route_top_p")
+    return idx, w
+
+
 def union(idx, E):
     idx = _c(idx, np.int32)
     T, k = idx.shape
@@ -136,6 +155,40 @@ def expert_ffn(x, H, F, expert, want_h=False):
     _check(lib().coli_oracle_expert_ffn(_p(x), H, F, *[_p(a) for a in arrs], _p(y), _p(h)),
            "expert_ffn")
     return (y, h) if want_h else y
+
+
+def _expert_tables(experts, E):
+    names = ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s")
+    keep, tables = [], []
+    for n in names:
+        arr = (ctypes.c_void_p * (E + 1))()
+        for e in range(E + 1):
+            if e in experts:
+                a = _c(experts[e][n], np.uint8 if n.endswith("_q") else np.float32)
+                keep.append(a)
+                arr[e] = a.ctypes.data
+            else:
+                arr[e] = None
+        tables.append(arr)
+    return keep, tables
+
+
+def moe_layer_top_p(x, H, F, E, k, routed_scale, top_p, w_router, sel_bias, experts):
+    """The layer with top-p routing.  Returns (idx, w, out [T,H] f64); dropped
+    slots have index -1 and weight 0."""
+    x = _c(widen(x), np.float64)
+    T = x.shape[0]
+    w_router = _c(w_router, np.float32); sel_bias = _c(sel_bias, np.float32)
+    keep, tables = _expert_tables(experts, E)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    out = np.empty((T, H), np.float64)
+    _check(lib().coli_oracle_moe_layer_top_p(_p(x), T, H, F, E, k, float(routed_scale), float(top_p),
+                                             _p(w_router), _p(sel_bias),
+                                             *[ctypes.cast(t, ctypes.c_void_p) for t in tables],
+                                             _p(idx), _p(w), _p(out)), "moe_layer_top_p")
+    del keep
+    return idx, w, out
 
 
 def moe_layer(x, H, F, E, k, routed_scale, w_router, sel_bias, experts):

@@ -257,3 +257,105 @@ int coli_oracle_moe_layer(const double* x, int64_t T, int64_t H, int64_t F,
     free(y);
     return 0;
 }
+
+/*
+ * Adaptive expert top-p ("colibri解説", section 速度を稼ぐ実用ノブ: the --topp 0.7
+ * knob, "adaptive expert top-p", which cuts expert reads by 30-40 %).  The page
+ * names the knob and its effect but not its rule; this library reads it as a
+ * cut of the routing distribution of the k experts the router selected:
+ *   pi_j = s_j / sum_j' s_j'            (unbiased sigmoids of the selected experts)
+ *   order the selected experts by pi descending (equal pi: lower expert first)
+ *   keep the shortest prefix of that order whose cumulative pi reaches top_p
+ *   (at least one expert; top_p >= 1 keeps all k)
+ *   w_j = routed_scale * s_j / sum_{kept} s     for kept experts (the router's
+ *         renormalisation, taken over the kept set)
+ * A dropped expert keeps its slot with index -1 and weight 0.
+ */
+int coli_oracle_route_top_p(const double* x, int64_t T, int64_t H,
+                            const float* w_router, const float* sel_bias, int64_t E, int64_t k,
+                            double routed_scale, double top_p, int32_t* topk_idx, double* topk_w)
+{
+    if (!x || !w_router || !sel_bias || !topk_idx || !topk_w) return -1;
+    if (T < 0 || H <= 0 || E <= 0 || k <= 0 || k > E || !(top_p > 0.0)) return -1;
+    double* sig = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * (size_t)E);
+    int64_t* order = (int64_t*)malloc(sizeof(int64_t) * (size_t)k);
+    char* keep = (char*)malloc((size_t)k);
+    if (!sig || !order || !keep) { free(sig); free(order); free(keep); return -1; }
+    int rc = coli_oracle_route(x, T, H, w_router, sel_bias, E, k, routed_scale, topk_idx, topk_w, NULL, sig, NULL);
+    if (rc != 0) { free(sig); free(order); free(keep); return rc; }
+    for (int64_t t = 0; t < T; ++t) {
+        int32_t* idx = topk_idx + t * k;
+        double* w = topk_w + t * k;
+        const double* st = sig + t * E;
+        double total = 0.0;
+        for (int64_t j = 0; j < k; ++j) total += st[idx[j]];
+        /* slots by pi descending, lower expert first on ties (selection sort) */
+        for (int64_t j = 0; j < k; ++j) { order[j] = j; keep[j] = 0; }
+        for (int64_t a = 0; a < k; ++a) {
+            int64_t best = a;
+            for (int64_t b = a + 1; b < k; ++b) {
+                const double sb = st[idx[order[b]]], sx = st[idx[order[best]]];
+                if (sb > sx || (sb == sx && idx[order[b]] < idx[order[best]])) best = b;
+            }
+            const int64_t tmp = order[a]; order[a] = order[best]; order[best] = tmp;
+        }
+        double cum = 0.0, kept = 0.0;
+        for (int64_t a = 0; a < k; ++a) {
+            keep[order[a]] = 1;
+            cum += st[idx[order[a]]] / total;
+            if (cum >= top_p) break;
+        }
+        for (int64_t j = 0; j < k; ++j)  /* the router's sum, in slot order, over the kept set */
+            if (keep[j]) kept += st[idx[j]];
+        for (int64_t j = 0; j < k; ++j) {
+            if (keep[j]) {
+                w[j] = routed_scale * st[idx[j]] / kept;
+            } else {
+                idx[j] = -1;
+                w[j] = 0.0;
+            }
+        }
+    }
+    free(sig); free(order); free(keep);
+    return 0;
+}
+
+/*
+ * The layer with adaptive expert top-p routing: out_t = sum over the kept
+ * slots of w[t,j] * FFN_{idx[t,j]}(x_t) + FFN_E(x_t).
+ */
+int coli_oracle_moe_layer_top_p(const double* x, int64_t T, int64_t H, int64_t F,
+                                int64_t E, int64_t k, double routed_scale, double top_p,
+                                const float* w_router, const float* sel_bias,
+                                const uint8_t* const* gate_q, const float* const* gate_s,
+                                const uint8_t* const* up_q, const float* const* up_s,
+                                const uint8_t* const* down_q, const float* const* down_s,
+                                int32_t* topk_idx, double* topk_w, double* out)
+{
+    if (!x || !gate_q || !gate_s || !up_q || !up_s || !down_q || !down_s) return -1;
+    if (!topk_idx || !topk_w || !out) return -1;
+    int rc = coli_oracle_route_top_p(x, T, H, w_router, sel_bias, E, k, routed_scale, top_p, topk_idx, topk_w);
+    if (rc != 0) return rc;
+    double* y = (double*)malloc(sizeof(double) * (size_t)H);
+    if (!y) return -1;
+    for (int64_t t = 0; t < T; ++t) {
+        const double* xt = x + t * H;
+        double* ot = out + t * H;
+        for (int64_t n = 0; n < H; ++n) ot[n] = 0.0;
+        for (int64_t j = 0; j <= k; ++j) {
+            const int64_t e = j < k ? topk_idx[t * k + j] : E;
+            if (e < 0) continue; /* dropped slot */
+            if (!gate_q[e] || !gate_s[e] || !up_q[e] || !up_s[e] || !down_q[e] || !down_s[e]) {
+                free(y);
+                return -1;
+            }
+            rc = coli_oracle_expert_ffn(xt, H, F, gate_q[e], gate_s[e], up_q[e], up_s[e],
+                                        down_q[e], down_s[e], y, NULL);
+            if (rc != 0) { free(y); return rc; }
+            const double wj = j < k ? topk_w[t * k + j] : 1.0;
+            for (int64_t n = 0; n < H; ++n) ot[n] += wj * y[n];
+        }
+    }
+    free(y);
+    return 0;
+}

@@ -89,6 +89,22 @@ int coli_oracle_moe_layer(const double* x, int64_t T, int64_t H, int64_t F,
 /* Number of threads the oracle's parallel loops use (1 without OpenMP). */
 int coli_oracle_threads(void);
 
+/* Adaptive expert top-p on top of coli_oracle_route (see coli_oracle.c):
+ * dropped slots get index -1 and weight 0; kept weights are renormalised over
+ * the kept experts.  top_p >= 1 gives coli_oracle_route's result. */
+int coli_oracle_route_top_p(const double* x, int64_t T, int64_t H,
+                            const float* w_router, const float* sel_bias, int64_t E, int64_t k,
+                            double routed_scale, double top_p, int32_t* topk_idx, double* topk_w);
+
+/* The layer with top-p routing (dropped slots contribute nothing). */
+int coli_oracle_moe_layer_top_p(const double* x, int64_t T, int64_t H, int64_t F,
+                                int64_t E, int64_t k, double routed_scale, double top_p,
+                                const float* w_router, const float* sel_bias,
+                                const uint8_t* const* gate_q, const float* const* gate_s,
+                                const uint8_t* const* up_q, const float* const* up_s,
+                                const uint8_t* const* down_q, const float* const* down_s,
+                                int32_t* topk_idx, double* topk_w, double* out);
+
 #ifdef __cplusplus
 }
 #endif
