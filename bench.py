@@ -41,18 +41,22 @@ NOMINAL_MS = {1: 0.06, 2: 0.3, 3: 3.0, 4: 5.0}
 TIMED_TARGET_S = 0.3  # aim for about this much timed work per workload
 
 
-def kernels_per_call(path, T, E):
-    """Our kernel launches in one layer call, by kernel chain: the one-token
-    chain runs router scores, top-k, gate/up, down and combine; the CUDA-core
-    decode chain runs router scores, top-k + union (one kernel up to 256
-    tokens), gate/up, down and combine; the prefill chain runs router scores,
-    (top-k,) union, the token-row gather, two grouped GEMMs and the slot sum."""
+def kernels_per_call(path, T, E, group_tokens=4):
+    """Our kernel launches in one layer call, by kernel chain: the fused
+    decode-layer kernel is one launch (plus the router-score kernel when the
+    batch has more tokens than one group); the prefill chain runs router
+    scores, top-k and union (one kernel up to 256 tokens, else the top-k and
+    three union kernels), the token-row gather, two grouped GEMMs and the slot
+    sum; the wide chain runs router scores, top-k + union, gate/up, down and
+    combine."""
     fused = T <= 256 and E <= 256
     if path == "single":
-        return 5
+        return 1
     if path == "decode":
+        return 1 if T <= group_tokens else 2
+    if path == "wide":
         return 5 if fused else 6
-    return 6 if fused else 7
+    return 6 if fused else 9
 
 
 def parse(argv=None):
@@ -67,6 +71,9 @@ def parse(argv=None):
     ap.add_argument("--experts", type=int, default=0,
                     help="routed experts per layer (0 = the workload's; profiling: fewer, same per-call bytes)")
     ap.add_argument("--replays", type=int, default=0, help="timed replays of the K steps (0 = sized to ~0.3 s)")
+    ap.add_argument("--top-p", type=float, default=0.0,
+                    help="also time decode batch 1 with adaptive expert top-p (0 = the default 0.7 entry only "
+                         "when all workloads run)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args(argv)
@@ -301,8 +308,9 @@ def traffic_from_profiles(kernel, workload):
 # the dominant kernel of each kernel chain, the stage whose events bracket it,
 # and the name of its committed ncu summary
 DOMINANT = {
-    "single": ("gateup_single_kernel", "gateup", "gateup"),
-    "decode": ("expert_phase_kernel<gateup>", "gateup", "gateup-phase"),
+    "single": ("moe_layer_kernel", "gateup", "layer"),
+    "decode": ("moe_layer_kernel", "gateup", "layer"),
+    "wide": ("expert_phase_kernel<gateup>", "gateup", "gateup-phase"),
     "prefill": ("prefill_gemm_kernel<gate/up>", "gateup", "prefill-gemm"),
 }
 
@@ -319,8 +327,9 @@ class Resident:
         self.H, self.F, self.E = c.H, c.F, c.E
 
 
-def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sampler_index):
-    """Time one workload; returns the fields of its benchmark entry."""
+def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sampler_index, top_p=0.0):
+    """Time one workload; returns the fields of its benchmark entry.  top_p > 0
+    runs the layer with adaptive expert top-p routing."""
     hbm_peak, bf16_peak, bf16_sust, peak_kind = peaks
     routers, layers = [], []
     for l in range(N_LAYERS):
@@ -329,7 +338,7 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         b = res.bufs[l]
         layers.append(coli.Layer(c.H, c.F, c.E, c.k, c.routed_scale, torch.from_numpy(w_router).cuda(),
                                  torch.from_numpy(sel_bias).cuda(), b["gate_q"], b["gate_s"], b["up_q"],
-                                 b["up_s"], b["down_q"], b["down_s"]))
+                                 b["up_s"], b["down_q"], b["down_s"], top_p=top_p))
     path = coli.moe_path(layers[0], c.T)
 
     # activation pool: G distinct (step, layer) batches, G a multiple of the layer count
@@ -432,7 +441,7 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
     stage_ms = {n: float(np.mean([ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]) for i in range(G)]))
                 for j, n in enumerate(STAGE_NAMES)}
     idx_all = idx_dev.cpu().numpy()
-    U = np.array([len(np.unique(idx_all[i])) for i in range(G)], np.float64)
+    U = np.array([len(np.unique(idx_all[i][idx_all[i] >= 0])) for i in range(G)], np.float64)  # top-p drops: -1
     gu_bytes_per_expert = 2 * (c.F * c.H // 2 + c.F * c.H // 64 * 4)
     x_bytes = c.T * c.H * (2 if c.x_dtype == "bf16" else 4)
     out_bytes = c.T * c.H * (2 if c.out_dtype == "bf16" else 4)
@@ -450,6 +459,18 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
                     "frac": gu_tflops / bf16_sust, "traffic": traffic,
                     "peak_kind": peak_kind + " (sustained bf16)", "alg_flops_per_launch": gu_flops,
                     "launch_ms": stage_ms[kstage]}
+    elif path in ("single", "decode"):
+        # the fused decode-layer kernel: every selected expert's int4 + scales, the
+        # router weights when it scores the tokens itself (T <= 4), activations, output
+        router_in_kernel = c.T <= 4
+        k_alg = float(np.mean((U + 1) * c.expert_bytes)) + x_bytes + out_bytes + \
+            (c.E * c.H * 4 + c.E * 4 if router_in_kernel else 0)
+        k_gbs = k_alg / (stage_ms[kstage] * 1e-3) / 1e9
+        roofline = {"kernel": kname + " (router" + (" scores, " if router_in_kernel else " top-k, ") +
+                    "union, gate/up + SwiGLU, down, weighted combine; one cooperative launch)",
+                    "bound": "hbm", "achieved": k_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": k_gbs / hbm_peak, "traffic": traffic, "peak_kind": peak_kind,
+                    "alg_bytes_per_launch": k_alg, "launch_ms": stage_ms[kstage]}
     else:
         gu_alg = float(np.mean((U + 1) * gu_bytes_per_expert)) + x_bytes
         gu_gbs = gu_alg / (stage_ms[kstage] * 1e-3) / 1e9
@@ -461,7 +482,8 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         alg = roofline.get("alg_bytes_per_launch")
         roofline["traffic_over_alg"] = traffic / alg if alg else None
     expert_alg = float(np.mean((U + 1) * c.expert_bytes))  # selected experts' int4 + scales only
-    entry = {"workload": workload_desc(c), "tokens_per_call": c.T, "path": path, "value": value,
+    entry = {"workload": workload_desc(c) + (f", adaptive expert top-p {top_p}" if top_p else ""),
+             "tokens_per_call": c.T, "path": path, "value": value, "top_p": top_p,
              "unit": "tokens/s", "steps": steps, "timed_replays": R, "ms_per_step": ms_per_step,
              "ms_per_step_p10": percentile(ms_max, 10) / steps, "ms_per_step_p90": percentile(ms_max, 90) / steps,
              "roofline": roofline, "gpu_launches": steps * kernels_per_call(path, c.T, c.E),
@@ -550,6 +572,12 @@ def run_ours(args):
         entries[k] = measure_workload(args, torch, coli, cfg_of(k), res, seed, world, rank, peaks,
                                       torch.cuda.current_device())
         torch.cuda.empty_cache()
+    topp = None
+    if not args.config or args.top_p:
+        # decode batch 1 with the pages' --topp 0.7 knob: fewer expert bytes per token
+        topp = measure_workload(args, torch, coli, cfg_of(1), res, seed, world, rank, peaks,
+                                torch.cuda.current_device(), top_p=args.top_p or 0.7)
+        torch.cuda.empty_cache()
 
     head_cfg = cfgs[0]
     head, c = entries[head_cfg], cfg_of(head_cfg)
@@ -561,8 +589,10 @@ def run_ours(args):
              "expert_alg_bytes_per_call": head["expert_alg_bytes_per_call"],
              "expert_frac_of_hbm_peak": head["expert_frac_of_hbm_peak"], "stage_ms": head["stage_ms"],
              "timing": "median of the timed replays of exactly K steps (CUDA events, max over ranks)"}
-    if len(cfgs) > 1:
+    if len(cfgs) > 1 or topp is not None:
         extra["per_workload"] = {cfg_of(k).name: entries[k] for k in cfgs[1:]}
+        if topp is not None:
+            extra["per_workload"][f"{cfg_of(1).name}-topp{topp['top_p']}"] = topp
     line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": head["steps"],
             "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,

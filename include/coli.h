@@ -77,6 +77,7 @@ typedef struct {
     const float* gate_s;   /* [E+1, F, H/64] */
     const float* up_s;     /* [E+1, F, H/64] */
     const float* down_s;   /* [E+1, H, F/64] */
+    float top_p;           /* adaptive expert top-p: 0 (or >= 1) = plain top-k; see coli_moe_forward */
 } coli_moe_layer;
 
 /*
@@ -117,15 +118,16 @@ COLI_API coli_status coli_expert_union(const int32_t* topk_idx, int T, int k, in
 COLI_API size_t coli_moe_workspace_size(const coli_moe_layer* layer, int T);
 
 /* Device status of a coli_moe_forward call (no counterpart on the pages: it
- * reports on this library's own kernels).  Kernels whose warps wait on one
- * another inside a launch bound every wait in time; a wait that runs out (a
- * fault or stall elsewhere on the GPU) leaves the outputs undefined and sets a
- * 32-bit status word in the workspace, which is 0 after a normal call.  This
- * returns the byte offset of that word inside the workspace of a call with T
- * tokens of this layer: read the 4 bytes after the call has completed (e.g. with
- * cudaMemcpy).  Returns SIZE_MAX if the sizes are invalid, if T == 0, or if a
- * call of this shape does not write the word (the one-token kernels have no such
- * waits).  Host arithmetic only: launches nothing, touches no device memory. */
+ * reports on this library's own kernels).  Kernels whose warps or blocks wait
+ * on one another inside a launch bound every wait in time; a wait that runs out
+ * (a fault or stall elsewhere on the GPU) leaves the outputs undefined and sets
+ * a 32-bit status word in the workspace, which is 0 after a normal call
+ * (1: a prefill GEMM pipeline wait ran out; 2: a decode-kernel grid barrier
+ * did; 3: the decode kernel was not launched cooperatively).  This returns the
+ * byte offset of that word inside the workspace of a call with T tokens of this
+ * layer: read the 4 bytes after the call has completed (e.g. with cudaMemcpy).
+ * Returns SIZE_MAX if the sizes are invalid or T == 0.  Host arithmetic only:
+ * launches nothing, touches no device memory. */
 COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
 
 /*
@@ -135,7 +137,15 @@ COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
  * The pages name the routed experts, the shared expert ("Colibri 完全ガイド",
  * DeepSeek-V3 router row) and int4 weights with one scale per 64; the SwiGLU
  * form of the expert and the unscaled, always-on shared expert are this
- * library's reading of them.  The router is fp32.  Batches of up to 64 tokens
+ * library's reading of them.
+ * Adaptive expert top-p (layer->top_p in (0, 1); "colibri解説", section 速度を稼ぐ
+ * 実用ノブ, the --topp knob, which the page credits with 30-40 % fewer expert
+ * reads): of the k selected experts, ranked by share s_j / sum s (descending,
+ * lower expert first), only the shortest prefix whose cumulative share reaches
+ * top_p is kept; the kept weights are renormalised to routed_scale over the
+ * kept experts, dropped slots are reported as index -1 with weight 0 and cost
+ * no expert reads.  The rule is this library's reading: the page names the
+ * knob and its effect only.  The router is fp32.  Batches of up to 64 tokens
  * compute the experts in fp32 (bf16 x is widened exactly); larger batches run
  * them on the tensor cores with bf16 operands (weights q * scale, activations
  * and the SwiGLU output rounded to bf16) and fp32 accumulation.  out is written
@@ -153,18 +163,22 @@ COLI_API coli_status coli_moe_forward(const coli_moe_layer* layer, const void* x
 /* Kernel chains of coli_moe_forward (coli_moe_path). */
 enum {
     COLI_PATH_NONE = 0,     /* empty batch or invalid arguments: nothing runs */
-    COLI_PATH_SINGLE = 1,   /* one token at hidden 6144, ffn 2048, <= 256 experts: the one-token chain */
-    COLI_PATH_DECODE = 2,   /* CUDA-core int4 GEMV kernels (fp32 arithmetic) */
-    COLI_PATH_PREFILL = 3   /* tcgen05 tensor-core grouped GEMMs (bf16 operands, fp32 accumulation) */
+    COLI_PATH_SINGLE = 1,   /* one token: the fused decode-layer kernel, down summed by output rows */
+    COLI_PATH_DECODE = 2,   /* 1-64 tokens: the fused decode-layer kernel (CUDA cores, fp32) */
+    COLI_PATH_PREFILL = 3,  /* > 64 tokens: tcgen05 tensor-core grouped GEMMs (bf16 operands, fp32 accumulation) */
+    COLI_PATH_WIDE = 4      /* batches neither kernel takes: CUDA-core expert-phase kernels (fp32) */
 };
 
 /*
  * Which kernel chain coli_moe_forward runs for a batch of T tokens of this
- * layer.  Decided by the shapes alone: more than 64 tokens with hidden and ffn
- * multiples of 256 take the tensor-core path (a device without
- * cuTensorMapEncodeTiled in its driver then gets COLI_ERR_UNSUPPORTED from
- * coli_moe_forward, never another path); every other valid batch runs on CUDA
- * cores in fp32.  Host-only, launches nothing.
+ * layer.  Decided by the shapes alone.  Batches of up to 64 tokens run the
+ * fused decode-layer kernel (one cooperative launch; with more than one token
+ * group it is preceded by the router-score kernel) when its shared memory
+ * (activations, union tables) fits in 227 KB; batches of more than 64 tokens
+ * with hidden and ffn multiples of 256 take the tensor-core path (a device
+ * without cuTensorMapEncodeTiled in its driver then gets COLI_ERR_UNSUPPORTED
+ * from coli_moe_forward, never another path); every other valid batch runs the
+ * CUDA-core expert-phase kernels in fp32.  Host-only, launches nothing.
  */
 COLI_API int coli_moe_path(const coli_moe_layer* layer, int T);
 
@@ -227,6 +241,31 @@ COLI_API coli_status coli_moe_forward_noalloc(const coli_moe_layer* layer, const
 
 COLI_API const char* coli_status_string(coli_status status);
 COLI_API const char* coli_last_error(void);
+
+/*
+ * Test hook, not part of the layer's interface.  Every wait inside the kernels
+ * (the decode kernel's grid barriers, the prefill GEMMs' pipeline waits) gives
+ * up after a time limit (2 s), records a non-zero status word
+ * (coli_moe_status_word_offset) and lets the kernel finish, so a stuck wait
+ * never hangs the GPU.  This call sets that limit for the launches that follow
+ * (ns = 0 restores the built-in limit), so that tests can make waits run out on
+ * purpose and check the status word; the outputs of such a call are undefined.
+ * Process-wide; teardown drains keep their own limits.
+ */
+COLI_API void coli_debug_set_wait_ns(unsigned long long ns);
+
+/*
+ * Test hook, not part of the layer's interface: the fused decode kernel runs
+ * its phases (router, union, gate/up, down, combine) inside one launch, where
+ * stream events cannot see them.  With a device buffer of at least
+ * (number of SMs) x 16 uint64 set here, the decode launches that follow record
+ * in it, per block, the GPU global timer (ns) at 16 fixed points of the kernel
+ * (0 start, 1 activations staged, 2 phase A done, 3 after the first grid
+ * barrier, 4 routing known, 5 gate/up done, 6 after the second barrier,
+ * 7 h staged, 8 down done, 9 end; unused points are left unwritten).  NULL
+ * turns it off.  Process-wide.
+ */
+COLI_API void coli_debug_phase_stamps(unsigned long long* device_buffer);
 
 #ifdef __cplusplus
 }

@@ -10,13 +10,14 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libcoli.so")
+# COLI_LIB=bounds loads the bounds-checked build (index checks write status 4 instead of trapping)
+LIB_PATH = os.path.join(PKG, "libcoli_bounds.so" if os.environ.get("COLI_LIB") == "bounds" else "libcoli.so")
 
 F32, BF16 = 0, 1
 STATUS = {0: "COLI_OK", 1: "COLI_ERR_INVALID_ARG", 2: "COLI_ERR_UNSUPPORTED", 3: "COLI_ERR_WORKSPACE",
           4: "COLI_ERR_CUDA"}
 STAGES = ("route", "union", "gateup", "down", "combine")
-PATHS = {0: "none", 1: "single", 2: "decode", 3: "prefill"}
+PATHS = {0: "none", 1: "single", 2: "decode", 3: "prefill", 4: "wide"}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
@@ -45,6 +46,10 @@ _lib.coli_status_string.restype = ctypes.c_char_p
 _lib.coli_status_string.argtypes = [_i]
 _lib.coli_last_error.restype = ctypes.c_char_p
 _lib.coli_last_error.argtypes = []
+_lib.coli_debug_set_wait_ns.restype = None
+_lib.coli_debug_set_wait_ns.argtypes = [ctypes.c_ulonglong]
+_lib.coli_debug_phase_stamps.restype = None
+_lib.coli_debug_phase_stamps.argtypes = [_p]
 
 
 class ColiError(RuntimeError):
@@ -58,7 +63,7 @@ class _LayerStruct(ctypes.Structure):
                 ("routed_scale", ctypes.c_float),
                 ("w_router", _p), ("sel_bias", _p),
                 ("gate_q", _p), ("up_q", _p), ("down_q", _p),
-                ("gate_s", _p), ("up_s", _p), ("down_s", _p)]
+                ("gate_s", _p), ("up_s", _p), ("down_s", _p), ("top_p", ctypes.c_float)]
 
 
 def lib():
@@ -102,7 +107,7 @@ class Layer:
     """One MoE layer: device tensors in the library's layout (expert E = shared)."""
 
     def __init__(self, hidden, ffn, n_experts, top_k, routed_scale, w_router, sel_bias,
-                 gate_q, gate_s, up_q, up_s, down_q, down_s, group=64):
+                 gate_q, gate_s, up_q, up_s, down_q, down_s, group=64, top_p=0.0):
         self.tensors = dict(w_router=w_router, sel_bias=sel_bias, gate_q=gate_q, gate_s=gate_s,
                             up_q=up_q, up_s=up_s, down_q=down_q, down_s=down_s)
         self.hidden, self.ffn, self.n_experts, self.top_k = hidden, ffn, n_experts, top_k
@@ -110,7 +115,7 @@ class Layer:
         self.struct = _LayerStruct(hidden, ffn, n_experts, top_k, group, routed_scale,
                                    *[_ptr(self.tensors[n]) for n in
                                      ("w_router", "sel_bias", "gate_q", "up_q", "down_q", "gate_s", "up_s",
-                                      "down_s")])
+                                      "down_s")], float(top_p))
 
     @property
     def ref(self):
@@ -136,8 +141,10 @@ def moe_workspace_size(layer, T):
 
 def moe_path(layer, T):
     """Name of the kernel chain moe_forward runs for T tokens of this layer:
-    "single" (one-token chain), "decode" (CUDA cores), "prefill" (tensor cores)
-    or "none" (empty or invalid call)."""
+    "single" (one token, fused decode-layer kernel), "decode" (fused
+    decode-layer kernel, up to 64 tokens), "prefill" (tensor cores), "wide"
+    (CUDA-core expert phases, for batches neither takes) or "none" (empty or
+    invalid call)."""
     return PATHS[int(_lib.coli_moe_path(layer.ref, T))]
 
 
@@ -177,3 +184,15 @@ def moe_profile_next(events):
 
 
 _prof_keep = None
+
+
+def debug_set_wait_ns(ns):
+    """Test hook: limit (ns) of the kernels' bounded waits for the launches that
+    follow; 0 restores the built-in limit.  See include/coli.h."""
+    _lib.coli_debug_set_wait_ns(int(ns))
+
+
+def debug_phase_stamps(buf):
+    """Test hook: record the decode kernel's per-block phase times into buf (a
+    torch int64 CUDA tensor of at least SMs x 16 elements), or stop (None)."""
+    _lib.coli_debug_phase_stamps(None if buf is None else buf.data_ptr())

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cmath>
 #include <cstdarg>
@@ -17,7 +18,7 @@
 #include "coli.h"
 #include "coli_common.cuh"
 #include "coli_decode.cuh"
-#include "coli_decode1.cuh"
+#include "coli_layer.cuh"
 #include "coli_prefill.cuh"
 #include "coli_router.cuh"
 #include "coli_union.cuh"
@@ -27,6 +28,17 @@ using namespace coli;
 namespace {
 
 thread_local char g_err[512] = "";
+
+// Test hook: device buffer for the decode kernel's per-CTA phase stamps (null = off).
+std::atomic<unsigned long long*> g_stamps{nullptr};
+
+// Test hook: limit of the kernels' bounded waits (0 = the built-in limits).
+std::atomic<unsigned long long> g_wait_ns{0};
+unsigned long long wait_limit(unsigned long long dflt)
+{
+    const unsigned long long v = g_wait_ns.load(std::memory_order_relaxed);
+    return v ? v : dflt;
+}
 thread_local cudaEvent_t* g_prof_events = nullptr;
 thread_local int g_prof_n = 0;
 
@@ -47,6 +59,9 @@ coli_status cuda_fail(cudaError_t e, const char* what)
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 constexpr int kMaxTokens = 65536;
+
+// Batches above this size take the tensor-core prefill path.
+constexpr int kDecodeMaxT = 64;
 
 coli_status check_sizes(int T, int H, int E, int k)
 {
@@ -69,6 +84,10 @@ DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
 constexpr int kMaxStageK = 16384;  // largest hidden / ffn width accepted
+
+// Dynamic shared memory the decode-layer kernel may use (it has no static shared
+// memory): sm_100's 227 KB per block, less 1 KB of slack.
+constexpr int kSmemBudget = 232448 - 1024;
 size_t gateup_smem(int H, int TG) { return stage_smem_bytes(H, TG); }
 size_t down_smem(int F, int TG) { return stage_smem_bytes(F, TG); }
 
@@ -76,6 +95,37 @@ template <typename Kern>
 cudaError_t allow_smem(Kern k, int bytes)
 {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// The fused decode-layer kernel, one instantiation per (tokens per group,
+// activation dtype, output dtype, one-token output-row mode).
+using LayerKernel = void (*)(const LayerArgs, const LayerSmem);
+LayerKernel layer_kernel(int MT, bool bf16, bool out_bf16, bool out_rows)
+{
+    if (MT == 4) {
+        if (bf16) return out_bf16 ? moe_layer_kernel<4, true, true, false> : moe_layer_kernel<4, true, false, false>;
+        return out_bf16 ? moe_layer_kernel<4, false, true, false> : moe_layer_kernel<4, false, false, false>;
+    }
+    if (out_rows) {
+        if (bf16) return out_bf16 ? moe_layer_kernel<1, true, true, true> : moe_layer_kernel<1, true, false, true>;
+        return out_bf16 ? moe_layer_kernel<1, false, true, true> : moe_layer_kernel<1, false, false, true>;
+    }
+    if (bf16) return out_bf16 ? moe_layer_kernel<1, true, true, false> : moe_layer_kernel<1, true, false, false>;
+    return out_bf16 ? moe_layer_kernel<1, false, true, false> : moe_layer_kernel<1, false, false, false>;
+}
+
+cudaError_t allow_layer_kernels(int bytes)
+{
+    const int mts[2] = {1, 4};
+    for (int mt : mts)
+        for (int rows = 0; rows < 2; ++rows)
+            for (int b = 0; b < 4; ++b) {
+                if (mt == 4 && rows) continue;
+                const cudaError_t e = cudaFuncSetAttribute(layer_kernel(mt, b & 1, b & 2, rows),
+                                                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+                if (e != cudaSuccess) return e;
+            }
+    return cudaSuccess;
 }
 
 coli_status device_info(DeviceInfo** out)
@@ -97,9 +147,7 @@ coli_status device_info(DeviceInfo** out)
             (e = allow_smem(expert_phase_kernel<true, true, 4>, lim)) != cudaSuccess ||
             (e = allow_smem(expert_phase_kernel<false, false, 1>, lim)) != cudaSuccess ||
             (e = allow_smem(expert_phase_kernel<false, false, 4>, lim)) != cudaSuccess ||
-            (e = allow_smem(gateup_single_kernel<false>, lim)) != cudaSuccess ||
-            (e = allow_smem(gateup_single_kernel<true>, lim)) != cudaSuccess ||
-            (e = allow_smem(down_single_kernel<0>, lim)) != cudaSuccess ||
+            (e = allow_layer_kernels(std::min(d.smem_optin, kSmemBudget))) != cudaSuccess ||  // no static smem
             (kPfSmemBytes <= (size_t)lim &&
              ((e = allow_smem(prefill_gemm_kernel<true>, (int)kPfSmemBytes)) != cudaSuccess ||
               (e = allow_smem(prefill_gemm_kernel<false>, (int)kPfSmemBytes)) != cudaSuccess)))
@@ -149,6 +197,8 @@ struct Workspace {
     int32_t* g_count;
     float* h;             // [P+T, F]
     float* partial;       // [P+T, H]
+    int32_t* chunk;       // [ceil(P / kUnionChunk), E] union bucket counts / starts (large batches)
+    int32_t* rank;        // [P] rank of each pair in its (chunk, expert) bucket
     size_t bytes;
 };
 
@@ -162,7 +212,8 @@ Workspace layout(void* base, int T, int H, int F, int E, int k)
         off += align_up(bytes, 256);
         return p;
     };
-    w.logits = (float*)take((size_t)T * E * 4);
+    // router scores [T, E]; up to 4 tokens the decode kernel writes per-piece partials [pieces, T, E]
+    w.logits = (float*)take((size_t)(T <= 4 ? stage_geom(H).per_lane : 1) * T * E * 4);
     w.idx = (int32_t*)take(P * 4);
     w.w = (float*)take(P * 4);
     w.count = (int32_t*)take((size_t)E * 4);
@@ -179,6 +230,9 @@ Workspace layout(void* base, int T, int H, int F, int E, int k)
     w.g_count = (int32_t*)take(G * 4);
     w.h = (float*)take(Q * F * 4);
     w.partial = (float*)take(Q * H * 4);
+    const bool big = T > kDecodeMaxT;  // the chunked union of large batches
+    w.chunk = (int32_t*)take(big ? (P + kUnionChunk - 1) / kUnionChunk * (size_t)E * 4 : 0);
+    w.rank = (int32_t*)take(big ? P * 4 : 0);
     w.bytes = off;
     return w;
 }
@@ -193,6 +247,7 @@ coli_status check_layer(const coli_moe_layer* L, int T)
     if (L->hidden > kMaxStageK || L->ffn > kMaxStageK)
         return fail(COLI_ERR_UNSUPPORTED, "hidden=%d / ffn=%d above %d", L->hidden, L->ffn, kMaxStageK);
     if (!std::isfinite(L->routed_scale)) return fail(COLI_ERR_INVALID_ARG, "routed_scale is not finite");
+    if (!(L->top_p >= 0.f) || !std::isfinite(L->top_p)) return fail(COLI_ERR_INVALID_ARG, "top_p is negative or not finite");
     const void* ptrs[] = {L->w_router, L->sel_bias, L->gate_q, L->up_q, L->down_q, L->gate_s, L->up_s, L->down_s};
     const char* names[] = {"w_router", "sel_bias", "gate_q", "up_q", "down_q", "gate_s", "up_s", "down_s"};
     for (int i = 0; i < 8; ++i) {
@@ -303,8 +358,6 @@ bool encode_weight_maps(CUtensorMap* q, CUtensorMap* s, const uint8_t* qp, const
                      CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Batches above this size take the tensor-core prefill path.
-constexpr int kDecodeMaxT = 64;
 
 // Batches up to this size take the top-k inside the union block.
 constexpr int kFusedTopkMaxT = 256;
@@ -312,12 +365,49 @@ constexpr int kFusedTopkMaxT = 256;
 // The kernel chain a valid call of T tokens runs (coli_moe_path), from the
 // shapes alone: every path's shared-memory needs fit the 227 KB per block of
 // sm_100, which the device set-up checks once.
+// The one-token output-row mode sizes its row buffer for GPUs of at least this many SMs.
+constexpr int kMinLayerSms = 64;
+
+// How the fused decode-layer kernel runs a batch: tokens per group (MT), the
+// one-token output-row mode, and its shared memory; ok = false if it does not fit.
+struct LayerPlan {
+    bool ok = false;
+    int MT = 1;
+    bool out_rows = false;
+    LayerSmem ls{};
+};
+
+LayerPlan layer_plan(int T, int H, int F, int E, int k)
+{
+    LayerPlan p;
+    if (T < 1 || T > kLayerMaxT) return p;
+    const int rows_per_cta = 2 * ((H / 2 + kMinLayerSms - 1) / kMinLayerSms);
+    auto fits = [&](int MT, bool rows) {
+        const LayerSmem ls = layer_smem(T, H, F, E, k, MT, rows, rows_per_cta);
+        if (ls.bytes > (size_t)kSmemBudget) return false;
+        p.ok = true;
+        p.MT = MT;
+        p.out_rows = rows;
+        p.ls = ls;
+        return true;
+    };
+    if (T == 1) {
+        if (fits(1, true) || fits(1, false)) return p;
+        return p;
+    }
+    if (fits(4, false) || fits(1, false)) return p;
+    return p;
+}
+
 int choose_path(const coli_moe_layer* L, int T)
 {
     if (T == 0) return COLI_PATH_NONE;
-    if (T == 1 && L->n_experts <= 256 && L->hidden == 1024 * 2 * kHalf && L->ffn == 2048) return COLI_PATH_SINGLE;
+    if (T <= kDecodeMaxT) {
+        const LayerPlan pl = layer_plan(T, L->hidden, L->ffn, L->n_experts, L->top_k);
+        if (pl.ok) return pl.out_rows ? COLI_PATH_SINGLE : COLI_PATH_DECODE;
+    }
     if (T > kDecodeMaxT && L->hidden % kPfRawK == 0 && L->ffn % kPfRawK == 0) return COLI_PATH_PREFILL;
-    return COLI_PATH_DECODE;
+    return COLI_PATH_WIDE;
 }
 
 }  // namespace
@@ -337,6 +427,10 @@ const char* coli_status_string(coli_status st)
 }
 
 const char* coli_last_error(void) { return g_err; }
+
+void coli_debug_set_wait_ns(unsigned long long ns) { g_wait_ns.store(ns, std::memory_order_relaxed); }
+
+void coli_debug_phase_stamps(unsigned long long* device_buffer) { g_stamps.store(device_buffer); }
 
 coli_status coli_moe_profile_next(cudaEvent_t* events, int n_events)
 {
@@ -400,8 +494,6 @@ int coli_moe_path(const coli_moe_layer* L, int T)
 size_t coli_moe_status_word_offset(const coli_moe_layer* L, int T)
 {
     if (check_layer(L, T) != COLI_OK || T == 0) return SIZE_MAX;
-    // the one-token chain runs no union kernel, which is what zeroes the word
-    if (choose_path(L, T) == COLI_PATH_SINGLE) return SIZE_MAX;
     char* const base = reinterpret_cast<char*>(256);  // any aligned base: only differences are used
     const Workspace w = layout(base, T, L->hidden, L->ffn, L->n_experts, L->top_k);
     return (size_t)(reinterpret_cast<char*>(w.ctl + 3) - base);
@@ -441,43 +533,45 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     // One token: router scores, top-k, gate/up, down, combine; the union of a
     // one-token batch is its k experts.
     const int path = choose_path(L, T);
-    const size_t s1_gu = stage_smem_bytes(H, 1), s1_dn = stage_smem_bytes(F, 1);
-    // (batch-1 path: see coli_decode1.cuh)
-    if (path == COLI_PATH_SINGLE) {
+
+    // Up to 64 tokens: the fused decode-layer kernel, one cooperative launch
+    // (after the router-score kernel when the batch is larger than one token group).
+    if (path == COLI_PATH_SINGLE || path == COLI_PATH_DECODE) {
+        const LayerPlan pl = layer_plan(T, H, F, E, k);
+        if (dev->sms < kMinLayerSms) return fail(COLI_ERR_UNSUPPORTED, "%d SMs: the decode kernel needs %d", dev->sms, kMinLayerSms);
+        const LayerKernel kern = layer_kernel(pl.MT, bf16, ot == COLI_BF16, pl.out_rows);
+        int occ = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, layer_threads(pl.MT), pl.ls.bytes)) != cudaSuccess)
+            return cuda_fail(e, "occupancy query");
+        if (occ < 1) return fail(COLI_ERR_UNSUPPORTED, "the decode kernel does not fit on an SM (%zu B shared memory)", pl.ls.bytes);
+        const bool fused_router = T <= pl.MT;
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
-        st = launch_logits(x, xt, 1, H, L->w_router, E, w.logits, nullptr, 0, stream);
-        if (st != COLI_OK) return st;
-        if ((e = launch_pdl(router_topk_kernel, 1, 32, 0, stream, (const float*)w.logits, 1, E, k, L->sel_bias,
-                            L->routed_scale, idx, wt)) != cudaSuccess)
-            return cuda_fail(e, "top-k launch");
+        if (!fused_router) {
+            st = launch_logits(x, xt, T, H, L->w_router, E, w.logits, nullptr, 0, stream);
+            if (st != COLI_OK) return st;
+        }
         if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess ||
             (e = tm.rec(COLI_STAGE_UNION, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_GATEUP, 0)) != cudaSuccess)
             return cuda_fail(e, "event record");
-        SingleArgs sa{L->gate_q, L->gate_s, L->up_q, L->up_s, L->down_q, L->down_s, H, F, E, k,
-                      L->routed_scale, w.logits, L->sel_bias, x, idx, wt, w.h, w.partial, out};
-        {
-            auto kern = bf16 ? gateup_single_kernel<true> : gateup_single_kernel<false>;
-            if ((e = launch_pdl(kern, dev->sms * blocks_per_sm(kern, s1_gu, kSingleThreads), kSingleThreads, s1_gu,
-                                stream, sa)) != cudaSuccess)
-                return cuda_fail(e, "gate/up launch");
-        }
-        if ((e = tm.rec(COLI_STAGE_GATEUP, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_DOWN, 0)) != cudaSuccess)
+        LayerArgs la{L->w_router, L->sel_bias, L->gate_q, L->gate_s, L->up_q, L->up_s, L->down_q, L->down_s,
+                     H, F, E, k, T, L->routed_scale, x, out, w.logits, fused_router ? 0 : 1, idx, wt, w.h,
+                     w.partial, w.ctl + 3, wait_limit(kBarrierNs), L->top_p, g_stamps.load()};
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(dev->sms);
+        cfg.blockDim = dim3(layer_threads(pl.MT));
+        cfg.dynamicSmemBytes = pl.ls.bytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, kern, la, pl.ls)) != cudaSuccess) return cuda_fail(e, "decode-layer launch");
+        // the layer kernel fuses gate/up, down and the combine
+        if ((e = tm.rec(COLI_STAGE_GATEUP, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_DOWN, 0)) != cudaSuccess ||
+            (e = tm.rec(COLI_STAGE_DOWN, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_COMBINE, 0)) != cudaSuccess ||
+            (e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess)
             return cuda_fail(e, "event record");
-        {
-            auto kern = down_single_kernel<0>;
-            if ((e = launch_pdl(kern, std::max(dev->sms * blocks_per_sm(kern, s1_dn, kSingleThreads), k + 1), kSingleThreads, s1_dn,
-                                stream, sa)) != cudaSuccess)
-                return cuda_fail(e, "down launch");
-        }
-        if ((e = tm.rec(COLI_STAGE_DOWN, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_COMBINE, 0)) != cudaSuccess)
-            return cuda_fail(e, "event record");
-        {
-            const int blocks = (H / 4 + 127) / 128;
-            e = ot == COLI_BF16 ? launch_pdl(combine_single_kernel<true>, blocks, 128, 0, stream, w.partial, k + 1, H, out)
-                                : launch_pdl(combine_single_kernel<false>, blocks, 128, 0, stream, w.partial, k + 1, H, out);
-            if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-        }
-        if ((e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
         e = cudaGetLastError();
         return e == cudaSuccess ? COLI_OK : cuda_fail(e, "layer launch");
     }
@@ -505,40 +599,45 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     if (path == COLI_PATH_PREFILL) {
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
         {
-            dim3 grid((T + kRtTile - 1) / kRtTile, (E + kRtTile - 1) / kRtTile);
-            if (bf16) router_logits_tiled_kernel<true><<<grid, 256, 0, stream>>>(x, T, H, L->w_router, E, w.logits);
-            else router_logits_tiled_kernel<false><<<grid, 256, 0, stream>>>(x, T, H, L->w_router, E, w.logits);
+            dim3 grid((T + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
+            if (bf16) router_logits_tiled_kernel<true><<<grid, kRtThreads, 0, stream>>>(x, T, H, L->w_router, E, w.logits);
+            else router_logits_tiled_kernel<false><<<grid, kRtThreads, 0, stream>>>(x, T, H, L->w_router, E, w.logits);
         }
         const bool fused = T <= kFusedTopkMaxT && E <= 256;
         if (!fused)
-            router_topk_kernel<<<(T + 7) / 8, 256, 0, stream>>>(w.logits, T, E, k, L->sel_bias, L->routed_scale, idx, wt);
+            router_topk_kernel<<<(T + 7) / 8, 256, 0, stream>>>(w.logits, T, E, k, L->sel_bias, L->routed_scale, L->top_p, idx, wt);
         if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess)
             return cuda_fail(e, "event record");
         WorkLists wl{w.pair_token, w.pair_w, w.ctl, w.g_expert, w.g_start, w.g_count, wt, kPfMaxN};
-        TopkArgs tk{w.logits, L->sel_bias, L->routed_scale, wt};
-        if (fused)
+        TopkArgs tk{w.logits, L->sel_bias, L->routed_scale, wt, L->top_p};
+        const int P = T * k;
+        if (fused) {
             union_kernel<true, true><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
                                                                       w.n_active, w.perm, w.inv_perm, wl, tk);
-        else
-            union_kernel<true, false><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
-                                                                       w.n_active, w.perm, w.inv_perm, wl, tk);
+        } else {  // the whole GPU: per-chunk ranks, bucket starts, scatter
+            const int n_chunks = (P + kUnionChunk - 1) / kUnionChunk;
+            union_chunk_kernel<<<n_chunks, kUnionChunk, 0, stream>>>(idx, P, E, w.chunk, w.rank);
+            union_scan_kernel<true><<<1, kUnionThreads, 0, stream>>>(w.chunk, n_chunks, T, k, E, w.count, w.offset,
+                                                                     w.active, w.n_active, wl);
+            union_scatter_kernel<true><<<(std::max(P, T) + 255) / 256, 256, 0, stream>>>(
+                idx, T, k, E, w.chunk, w.rank, w.offset, w.perm, w.inv_perm, wl);
+        }
         if ((e = tm.rec(COLI_STAGE_UNION, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_GATEUP, 0)) != cudaSuccess)
             return cuda_fail(e, "event record");
-        const int P = T * k;
         const int max_tiles = P / kPfMaxN + E + (T + kPfMaxN - 1) / kPfMaxN + 1;  // >= number of union groups
         {
             const size_t n = Q * (size_t)(H / 8);
             const int blocks = (int)((n + 255) / 256);
-            if (bf16) prefill_gather_kernel<true><<<blocks, 256, 0, stream>>>(x, w.pair_token, (int)Q, H, xg);
-            else prefill_gather_kernel<false><<<blocks, 256, 0, stream>>>(x, w.pair_token, (int)Q, H, xg);
+            if (bf16) prefill_gather_kernel<true><<<blocks, 256, 0, stream>>>(x, w.pair_token, (int)Q, T, H, xg);
+            else prefill_gather_kernel<false><<<blocks, 256, 0, stream>>>(x, w.pair_token, (int)Q, T, H, xg);
         }
-        PrefillArgs pa{F, H, k, P, F / 64, w.ctl, w.g_expert, w.g_start, w.g_count, w.perm, w.pair_w, hb, xg, w.ctl + 3};
+        PrefillArgs pa{F, H, k, P, F / 64, w.ctl, w.g_expert, w.g_start, w.g_count, w.perm, w.pair_w, hb, xg, w.ctl + 3, wait_limit(kPfWaitNs)};
         const int grid1 = std::min(dev->sms, max_tiles * (F / 64));
         prefill_gemm_kernel<true><<<grid1, kPfThreads, kPfSmemBytes, stream>>>(m_gq, m_uq, m_gs, m_us, m_x, pa);
         if ((e = tm.rec(COLI_STAGE_GATEUP, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_DOWN, 0)) != cudaSuccess)
             return cuda_fail(e, "event record");
         uint16_t* ys = xg;  // the gathered rows are dead once gate/up is done
-        PrefillArgs pd{H, F, k, P, H / 128, w.ctl, w.g_expert, w.g_start, w.g_count, w.perm, w.pair_w, hb, ys, w.ctl + 3};
+        PrefillArgs pd{H, F, k, P, H / 128, w.ctl, w.g_expert, w.g_start, w.g_count, w.perm, w.pair_w, hb, ys, w.ctl + 3, wait_limit(kPfWaitNs)};
         const int grid2 = std::min(dev->sms, max_tiles * (H / 128));
         prefill_gemm_kernel<false><<<grid2, kPfThreads, kPfSmemBytes, stream>>>(m_dq, m_dq, m_ds, m_ds, m_h, pd);
         if ((e = tm.rec(COLI_STAGE_DOWN, 1)) != cudaSuccess || (e = tm.rec(COLI_STAGE_COMBINE, 0)) != cudaSuccess)
@@ -546,8 +645,8 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
         {
             const size_t n8 = (size_t)T * H / 8;
             const int blocks = (int)((n8 + 255) / 256);
-            if (ot == COLI_BF16) slot_reduce_kernel<true><<<blocks, 256, 0, stream>>>(ys, T, k + 1, H, out);
-            else slot_reduce_kernel<false><<<blocks, 256, 0, stream>>>(ys, T, k + 1, H, out);
+            if (ot == COLI_BF16) slot_reduce_kernel<true><<<blocks, 256, 0, stream>>>(ys, T, k + 1, H, idx, out);
+            else slot_reduce_kernel<false><<<blocks, 256, 0, stream>>>(ys, T, k + 1, H, idx, out);
         }
         if ((e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
         e = cudaGetLastError();
@@ -562,13 +661,13 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     if (st != COLI_OK) return st;
     const bool fused_topk = T <= kFusedTopkMaxT && E <= 256;
     if (!fused_topk)
-        router_topk_kernel<<<(T + 7) / 8, 256, 0, stream>>>(w.logits, T, E, k, L->sel_bias, L->routed_scale, idx, wt);
+        router_topk_kernel<<<(T + 7) / 8, 256, 0, stream>>>(w.logits, T, E, k, L->sel_bias, L->routed_scale, L->top_p, idx, wt);
     if ((e = tm.rec(COLI_STAGE_ROUTE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
 
     // Union and work lists
     if ((e = tm.rec(COLI_STAGE_UNION, 0)) != cudaSuccess) return cuda_fail(e, "event record");
     WorkLists wl{w.pair_token, w.pair_w, w.ctl, w.g_expert, w.g_start, w.g_count, wt, TG};
-    TopkArgs tk{w.logits, L->sel_bias, L->routed_scale, wt};
+    TopkArgs tk{w.logits, L->sel_bias, L->routed_scale, wt, L->top_p};
     if (fused_topk)
         union_kernel<true, true><<<1, kUnionThreads, 0, stream>>>(idx, T, k, E, w.count, w.offset, w.active,
                                                                   w.n_active, w.perm, w.inv_perm, wl, tk);
@@ -607,8 +706,8 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     {
         const int n = T * (H / 4);
         const int blocks = (n + 255) / 256;
-        if (ot == COLI_BF16) combine_kernel<true><<<blocks, 256, 0, stream>>>(w.partial, w.inv_perm, T, k, H, out);
-        else combine_kernel<false><<<blocks, 256, 0, stream>>>(w.partial, w.inv_perm, T, k, H, out);
+        if (ot == COLI_BF16) combine_kernel<true><<<blocks, 256, 0, stream>>>(w.partial, w.inv_perm, idx, T, k, H, out);
+        else combine_kernel<false><<<blocks, 256, 0, stream>>>(w.partial, w.inv_perm, idx, T, k, H, out);
     }
     if ((e = tm.rec(COLI_STAGE_COMBINE, 1)) != cudaSuccess) return cuda_fail(e, "event record");
 

@@ -75,4 +75,39 @@ __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("grid
 
 __host__ __device__ __forceinline__ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Index checks of the bounds-checked build (libcoli_bounds.so, compiled with
+// COLI_DEBUG_BOUNDS): a failed check records status 4 in the call's status word
+// and the caller skips the access; nothing traps.  In the normal build the
+// check is the constant true and costs nothing.
+#ifdef COLI_DEBUG_BOUNDS
+__device__ __forceinline__ bool coli_in_bounds(bool ok, int* status)
+{
+    if (!ok && status) atomicExch(status, 4);
+    return ok;
+}
+#define COLI_IN_BOUNDS(cond, status) ::coli::coli_in_bounds((cond), (status))
+#else
+#define COLI_IN_BOUNDS(cond, status) true
+#endif
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Asynchronous global -> shared copies (cp.async): 16 bytes bypassing L1, 4 bytes
+// through L1; completion is tracked per thread in commit groups.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's most recent commit groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 }  // namespace coli

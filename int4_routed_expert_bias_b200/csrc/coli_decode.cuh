@@ -199,9 +199,10 @@ expert_phase_kernel(PhaseArgs a)
 
 // out[t, n] = sum_j partial[inv_perm[t*k + j], n] + partial[P + t, n], in slot
 // order j = 0..k-1, then the shared expert.  4 outputs per thread.
+// Slots whose routing index is -1 (dropped by adaptive top-p) are skipped.
 template <bool kOutBf16>
 __global__ void combine_kernel(const float* __restrict__ partial, const int32_t* __restrict__ inv_perm,
-                               int T, int k, int H, void* __restrict__ out)
+                               const int32_t* __restrict__ topk_idx, int T, int k, int H, void* __restrict__ out)
 {
     const int P = T * k;
     const int per_row = H / 4;
@@ -211,6 +212,7 @@ __global__ void combine_kernel(const float* __restrict__ partial, const int32_t*
     const int n = (i - t * per_row) * 4;
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
+        if (topk_idx[(size_t)t * k + j] < 0) continue;
         const int pos = inv_perm[(size_t)t * k + j];
         const float4 v = *reinterpret_cast<const float4*>(partial + (size_t)pos * H + n);
         s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;

@@ -130,44 +130,71 @@ __host__ __device__ inline size_t stage_smem_bytes(int K, int n_vectors)
 }
 
 // Stage n vectors; load(t, i) returns values i..i+3 of vector t (fp32).
-// All threads of the block call this (it uses warp shuffles).
+// Threads tid = 0 .. nthr-1 (whole warps) share the work; each has kU loads in
+// flight before it stores.  All nthr threads must call this (it uses warp
+// shuffles).
+template <typename Load4>
+__device__ __forceinline__ void stage_vectors_part(int n, Load4 load, const StageGeom& g, float4* xs, float* corr,
+                                                   int tid, int nthr)
+{
+    constexpr int kU = 8;
+    const int total = n * g.nch * 8;
+    for (int base = 0; base < total; base += kU * nthr) {
+        float4 v[kU];
+#pragma unroll
+        for (int r = 0; r < kU; ++r) {
+            const int idx = base + r * nthr + tid;
+            v[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (idx < total) {
+                const int t = idx / (g.nch * 8);
+                const int rem = idx - t * g.nch * 8;
+                v[r] = load(t, (rem >> 3) * kChunkK + (rem & 7) * 4);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kU; ++r) {
+            const int idx = base + r * nthr + tid;
+            const bool valid = idx < total;
+            int t = 0, c = 0, j = 0;
+            if (valid) {
+                t = idx / (g.nch * 8);
+                const int rem = idx - t * g.nch * 8;
+                c = rem >> 3;
+                j = rem & 7;
+                xs[(size_t)t * g.f4 + ((c >> 5) * 8 + j) * 32 + ((c & 31) ^ j)] =
+                    make_float4(v[r].y, v[r].x, v[r].w, v[r].z);
+            }
+            float odd = v[r].y + v[r].w, even = v[r].x + v[r].z;
+            odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 1);
+            even += __shfl_xor_sync(0xFFFFFFFFu, even, 1);
+            odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 2);
+            even += __shfl_xor_sync(0xFFFFFFFFu, even, 2);
+            odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 4);
+            even += __shfl_xor_sync(0xFFFFFFFFu, even, 4);
+            if (valid && j == 0) corr[t * g.nch + c] = fmaf(-24.f, odd, -264.f * even);
+        }
+    }
+}
+
+// The same with every thread of the block.
 template <typename Load4>
 __device__ __forceinline__ void stage_vectors_fn(int n, Load4 load, const StageGeom& g, float4* xs, float* corr)
 {
-    const int total = n * g.nch * 8;
-    for (int base = 0; base < total; base += blockDim.x) {
-        const int idx = base + threadIdx.x;
-        const bool valid = idx < total;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        int t = 0, c = 0, j = 0;
-        if (valid) {
-            t = idx / (g.nch * 8);
-            const int rem = idx - t * g.nch * 8;
-            c = rem >> 3;
-            j = rem & 7;
-            v = load(t, c * kChunkK + j * 4);
-            xs[(size_t)t * g.f4 + ((c >> 5) * 8 + j) * 32 + ((c & 31) ^ j)] = make_float4(v.y, v.x, v.w, v.z);
-        }
-        float odd = v.y + v.w, even = v.x + v.z;
-        odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 1);
-        even += __shfl_xor_sync(0xFFFFFFFFu, even, 1);
-        odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 2);
-        even += __shfl_xor_sync(0xFFFFFFFFu, even, 2);
-        odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 4);
-        even += __shfl_xor_sync(0xFFFFFFFFu, even, 4);
-        if (valid && j == 0) corr[t * g.nch + c] = fmaf(-24.f, odd, -264.f * even);
-    }
+    stage_vectors_part(n, load, g, xs, corr, (int)threadIdx.x, (int)blockDim.x);
 }
 
 // Stage n vectors; vector v is row rows(v) of src (K values each, fp32 or bf16).
 template <bool kBf16, typename RowOf>
 __device__ __forceinline__ void stage_vectors(const void* __restrict__ src, int K, int n, RowOf rows,
-                                              const StageGeom& g, float4* xs, float* corr)
+                                              const StageGeom& g, float4* xs, float* corr, int tid = -1,
+                                              int nthr = 0)
 {
     const size_t row_bytes = (size_t)K * (kBf16 ? 2 : 4);
-    stage_vectors_fn(n, [&](int t, int i) {
+    auto load = [&](int t, int i) {
         return load_act4<kBf16>(static_cast<const char*>(src) + (size_t)rows(t) * row_bytes, i);
-    }, g, xs, corr);
+    };
+    if (tid < 0) stage_vectors_fn(n, load, g, xs, corr);
+    else stage_vectors_part(n, load, g, xs, corr, tid, nthr);
 }
 
 }  // namespace coli

@@ -1,0 +1,1338 @@
+// coli_layer.cuh -- the whole MoE layer for decode batches (1..64 tokens) in one
+// cooperative launch: Route, Union, gate/up + SwiGLU, down and the weighted
+// combine, separated by grid-wide barriers.
+//
+// The pages' per-token path is Route -> Union -> expert compute (Korean
+// getting-started page, section 토큰당 처리 경로); the router is DeepSeek-V3's
+// sigmoid router with a selection bias ("Colibri 完全ガイド", section コア技術の
+// ハイライト) and the experts are int4 with one scale per 64 ("colibri: 744B MoE
+// …", section はじめにとソースが語らないこと); decode runs in fp32 (完全ガイド,
+// section 詳細解説 step 3).
+//
+// One CTA per SM, every CTA resident (cooperative launch).  Phases:
+//   A  router partial scores (fp32 weights x staged activations) and the
+//      shared expert's gate/up rows, which need no routing;
+//   -- grid barrier --
+//   B  every CTA takes the top-k of every token and the batch union (a stable
+//      counting sort in shared memory: the same result in every CTA); then the
+//      routed experts' gate/up rows.  With several tokens, also the shared
+//      expert's down rows.  One token: the shared expert's down rows for this
+//      CTA's output rows run while warp 0 takes the top-k;
+//   -- grid barrier --
+//   C  one token: this CTA's output rows of every selected down matrix, summed
+//      in slot order into out (no partial buffer, no further barrier).
+//      Several tokens: the routed down rows, one partial output per pair;
+//   -- grid barrier (several tokens) --
+//   D  several tokens: out[t] = sum over the token's slots (slot order) of the
+//      partial outputs, plus the shared expert's.
+//
+// Work inside a phase is a flat list of items (a gate/up row pair of one token
+// group, a down row pair, a router row piece) cut into contiguous, equally
+// costly ranges, one per CTA, and dealt to the CTA's warps round-robin; each
+// warp streams its items' int4 rows through a rolling register pipeline (the
+// loads of the next P chunk-steps are in flight while one is computed).  Each
+// int4 word is decoded once and applied to every token of the group.
+//
+// The only waits are the grid barriers; each gives up after a time limit,
+// records an error in the status word and lets the kernel finish.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "coli_int4.cuh"
+#include "coli_router.cuh"
+
+namespace coli {
+
+// Threads per block: 16 warps for one-token groups, 12 for four-token groups
+// (whose multiply-adds over four activation vectors need more registers).
+__host__ __device__ constexpr int layer_threads(int MT) { return MT == 1 ? 512 : 384; }
+constexpr int kLayerMaxT = 64;      // tokens (64-bit token masks in the union)
+constexpr unsigned long long kBarrierNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+
+// ---------------------------------------------------------------------------
+// grid barrier
+
+__device__ __forceinline__ unsigned long long layer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Barrier over all CTAs of a cooperative launch, on the launch's own barrier
+// word (zero-based, provided by the driver for cooperative launches).  CTA 0
+// adds 2^31 - (G - 1) and every other CTA 1, so bit 31 of the word flips
+// exactly when the last CTA arrives and the low bits return to where they
+// were.  Arrival releases and the poll acquires at GPU scope, so writes before
+// the barrier are visible after it.  Gives up after the deadline (error word
+// set) instead of waiting forever.
+__device__ __forceinline__ void grid_barrier(unsigned int* word, unsigned long long deadline, int* err)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned int add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+        unsigned int old, cur;
+        asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(word), "r"(add) : "memory");
+        while (true) {
+            asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(word) : "memory");
+            if ((old ^ cur) & 0x80000000u) break;
+            if (layer_ns() > deadline) {
+                atomicExch(err, 2);
+                break;
+            }
+            __nanosleep(64);
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// the rolling int4 row-pair engine
+
+// Two int4 rows (bytes and scales) that one item streams.
+struct RowPair {
+    const uint8_t* q0;
+    const uint8_t* q1;
+    const float* s0;
+    const float* s1;
+};
+
+// The staged vectors (offsets of their float4 slots, and of their chunk
+// corrections) that one item multiplies its rows with.
+template <int MT>
+struct VecSet {
+    int m;         // vectors used (<= MT)
+    int x4[MT];    // float4 slot offset of vector t
+    int cr[MT];    // correction offset of vector t
+};
+
+// One 16-byte chunk of both rows against up to MT staged vectors: each packed
+// word of each row is decoded once and applied to every vector.
+// xrow = the staged slots of this lane's chunk row block; off = swizzle offsets.
+template <int MT>
+__device__ __forceinline__ void chunk_pair_vectors(const uint4& w0, const uint4& w1, const float4* xrow,
+                                                   const VecSet<MT>& v, int lane, float2 (&acc)[2][MT])
+{
+#pragma unroll
+    for (int t = 0; t < MT; ++t) acc[0][t] = acc[1][t] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t a = q == 0 ? w0.x : q == 1 ? w0.y : q == 2 ? w0.z : w0.w;
+        const uint32_t b = q == 0 ? w1.x : q == 1 ? w1.y : q == 2 ? w1.z : w1.w;
+        const float2 a0 = nib_pair(a << 15), a1 = nib_pair(a << 7), a2 = nib_pair(a >> 1), a3 = nib_pair(a >> 9);
+        const float2 b0 = nib_pair(b << 15), b1 = nib_pair(b << 7), b2 = nib_pair(b >> 1), b3 = nib_pair(b >> 9);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            if (t < v.m) {
+                const float4 xlo = xrow[v.x4[t] + (2 * q) * 32 + (lane ^ (2 * q))];
+                const float4 xhi = xrow[v.x4[t] + (2 * q + 1) * 32 + (lane ^ (2 * q + 1))];
+                const float2 p0 = make_float2(xlo.x, xlo.y), p1 = make_float2(xlo.z, xlo.w);
+                const float2 p2 = make_float2(xhi.x, xhi.y), p3 = make_float2(xhi.z, xhi.w);
+                acc[0][t] = __ffma2_rn(a0, p0, acc[0][t]);
+                acc[1][t] = __ffma2_rn(b0, p0, acc[1][t]);
+                acc[0][t] = __ffma2_rn(a1, p1, acc[0][t]);
+                acc[1][t] = __ffma2_rn(b1, p1, acc[1][t]);
+                acc[0][t] = __ffma2_rn(a2, p2, acc[0][t]);
+                acc[1][t] = __ffma2_rn(b2, p2, acc[1][t]);
+                acc[0][t] = __ffma2_rn(a3, p3, acc[0][t]);
+                acc[1][t] = __ffma2_rn(b3, p3, acc[1][t]);
+            }
+        }
+    }
+}
+
+// Streams items j0, j0 + js, ... (nj of them) of a row-pair list: item j has
+// two int4 rows of K = 32 * nch values (rows_of(j, RowPair&)) and up to MT
+// staged vectors (vecs_of(j, VecSet&)).  The lane takes chunks c = lane + 32 i,
+// i < per_lane; a step is one chunk of both rows (16 bytes of each and their
+// two scales).  The steps' bytes travel through this warp's ring of R slots in
+// shared memory, filled by cp.async R - 1 steps ahead of the one being
+// computed, so the bytes in flight do not cost registers and the loop stays
+// small (the slot index is an address, not a register name).  At the end of
+// item j, finish(j, VecSet, tot) gets the lane's partial sums tot[row][vector]
+// (to be summed over the warp).  xs: staged float4 slots; corr: staged chunk
+// corrections; ring: this warp's R * kSlotBytes bytes.
+struct NoHook {
+    __device__ void operator()() const {}
+};
+
+constexpr int kSlotBytes = 32 * (16 + 16 + 4 + 4);  // one step of a warp: two 16-byte chunks and two scales per lane
+
+// hook(): called by every thread once the first R - 1 steps are in flight and
+// before the first one is consumed (e.g. a barrier and the staging of the
+// vectors), also by warps that have no items.
+__device__ __forceinline__ void cp_async16_s(uint32_t smem, const void* gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4_s(uint32_t smem, const void* gmem)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t smem)
+{
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(smem));
+    return r;
+}
+__device__ __forceinline__ float lds32(uint32_t smem)
+{
+    float r;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(smem));
+    return r;
+}
+
+template <int MT, int R, typename RowsOf, typename VecsOf, typename Finish, typename Hook = NoHook>
+__device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per_lane, int nch, const float4* xs,
+                                                 const float* corr, unsigned char* ring, RowsOf rows_of,
+                                                 VecsOf vecs_of, Finish finish, Hook hook = Hook())
+{
+    if (nj <= 0) {
+        hook();
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    const bool whole = (nch & 31) == 0;  // every lane has a chunk at every step
+    // this lane's bytes of ring slot 0 (16-byte chunk of row 0 at +0, of row 1 at +512; scales at sc_off, +128)
+    const uint32_t ring_lane = smem_u32(ring) + lane * 16;
+    const uint32_t ring_end = ring_lane + R * kSlotBytes;
+    const uint32_t sc_off = 1024 - 12 * lane;
+    // load cursor: item lj (0-based among mine), chunk step lci, this lane's slot address and source pointers
+    int lj = 0, lci = 0;
+    uint32_t lsl = ring_lane;
+    const uint8_t *pq0, *pq1;
+    const float *ps0, *ps1;
+    auto set_rows = [&](int j) {
+        RowPair r;
+        rows_of(j, r);
+        pq0 = r.q0 + lane * 16;
+        pq1 = r.q1 + lane * 16;
+        ps0 = r.s0 + (lane >> 1);
+        ps1 = r.s1 + (lane >> 1);
+    };
+    set_rows(j0);
+    auto issue = [&]() {
+        if (lj < nj && (whole || lane + 32 * lci < nch)) {
+            cp_async16_s(lsl, pq0);
+            cp_async16_s(lsl + 512, pq1);
+            cp_async4_s(lsl + sc_off, ps0);
+            cp_async4_s(lsl + sc_off + 128, ps1);
+        }
+        cp_async_commit();  // one group per step (empty past the end)
+        pq0 += 512;         // this lane's next chunk: 32 chunks on
+        pq1 += 512;
+        ps0 += 16;
+        ps1 += 16;
+        lsl += kSlotBytes;
+        if (lsl == ring_end) lsl = ring_lane;
+        if (++lci == per_lane) {
+            lci = 0;
+            if (++lj < nj) set_rows(j0 + lj * js);
+        }
+    };
+#pragma unroll 1
+    for (int u = 0; u < R - 1; ++u) issue();
+    hook();
+
+    int cj = 0, cci = 0;
+    uint32_t csl = ring_lane;
+    VecSet<MT> v;
+    vecs_of(j0, v);
+    float tot[2][MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
+    const float4* xrow = xs;
+    const float* crow = corr + lane;
+    const int S = nj * per_lane;
+#pragma unroll 1
+    for (int s = 0; s < S; ++s) {
+        issue();                   // step s + R - 1 into the slot consumed last iteration
+        cp_async_wait<R - 1>();    // step s has landed (this lane's own bytes)
+        if (whole || lane + 32 * cci < nch) {
+            const uint4 w0 = lds128(csl), w1 = lds128(csl + 512);
+            const float s0 = lds32(csl + sc_off), s1 = lds32(csl + sc_off + 128);
+            float2 acc[2][MT];
+            chunk_pair_vectors<MT>(w0, w1, xrow, v, lane, acc);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                if (t < v.m) {
+                    const float cr = crow[v.cr[t]];
+                    tot[0][t] = chunk_finish(acc[0][t], cr, s0, tot[0][t]);
+                    tot[1][t] = chunk_finish(acc[1][t], cr, s1, tot[1][t]);
+                }
+            }
+        }
+        csl += kSlotBytes;
+        if (csl == ring_end) csl = ring_lane;
+        xrow += 256;
+        crow += 32;
+        if (++cci == per_lane) {
+            cci = 0;
+            xrow = xs;
+            crow = corr + lane;
+            finish(j0 + cj * js, v, tot);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
+            if (++cj < nj) vecs_of(j0 + cj * js, v);
+        }
+    }
+    cp_async_wait<0>();  // the trailing (empty) groups: nothing is left in flight into the ring
+}
+
+// ---------------------------------------------------------------------------
+// layer arguments and shared-memory layout
+
+struct LayerArgs {
+    const float* w_router;  // [E, H]
+    const float* sel_bias;  // [E]
+    const uint8_t* gate_q;
+    const float* gate_s;
+    const uint8_t* up_q;
+    const float* up_s;
+    const uint8_t* down_q;
+    const float* down_s;
+    int H, F, E, k, T;
+    float routed_scale;
+    const void* x;          // [T, H] fp32 or bf16
+    void* out;              // [T, H] fp32 or bf16
+    float* logit_part;      // [n_pieces, T, E] router partial scores (n_pieces = 1: computed before the launch)
+    int n_pieces;           // 0: the kernel computes the router (pieces of 1024 K); else precomputed pieces
+    int32_t* idx_out;       // [T, k]
+    float* w_out;           // [T, k]
+    float* h;               // [T*k + T, F] SwiGLU outputs, sorted pair order, shared expert at T*k + t
+    float* y;               // [T*k + T, H] partial outputs (several tokens)
+    int* err;               // status word
+    unsigned long long wait_ns;  // limit of each grid-barrier wait
+    float top_p;            // adaptive expert top-p (0: plain top-k)
+    unsigned long long* stamps;  // optional [gridDim.x, kStamps] globaltimer stamps per CTA (test hook)
+};
+
+constexpr int kStamps = 16;
+
+// Test hook: thread 0 of each CTA records the time it reached point i.
+__device__ __forceinline__ void stamp(const LayerArgs& a, int i)
+{
+    if (a.stamps && threadIdx.x == 0) a.stamps[blockIdx.x * kStamps + i] = layer_ns();
+}
+
+// Shared-memory plan of one launch (host and device compute the same one).
+// The union tables' offsets are kernel parameters, so their addresses are one
+// add away and need no registers across the kernel.
+struct LayerSmem {
+    int nx;       // activation vectors staged (all tokens when T <= MT, else MT)
+    int nh;       // h vectors staged
+    size_t x_off, h_off, u_off, y_off, bytes;
+    // union tables (byte offsets from the start of shared memory)
+    uint32_t mask, cnt, off, gpre, idx, w, perm, ipos, gexp, gpos, seg_c, seg_i, seg_cost, tmp;
+    uint32_t logit;  // router scores [T, E] of the tokens (when the kernel scores them itself)
+    uint32_t ring;   // the warps' cp.async rings, warps x ring_slots x kSlotBytes
+    int ring_slots;
+};
+
+// Ring slots per warp: deeper when fewer activation vectors are staged.
+__host__ __device__ constexpr int layer_ring_slots(int MT) { return MT == 1 ? 5 : 4; }
+
+// rows_per_cta: output rows of one CTA in the one-token output-row mode.
+__host__ __device__ inline LayerSmem layer_smem(int T, int H, int F, int E, int k, int MT, bool out_rows,
+                                                int rows_per_cta)
+{
+    LayerSmem s{};
+    s.nx = T <= MT ? T : MT;
+    s.nh = out_rows ? k + 1 : MT;
+    size_t off = 0;
+    s.x_off = off;
+    off += align_up(stage_smem_bytes(H, s.nx), 16);
+    s.h_off = off;
+    off += align_up(stage_smem_bytes(F, s.nh), 16);
+    s.u_off = off;
+    {
+        const size_t P = (size_t)T * k;
+        size_t o = off;
+        auto take = [&](size_t bytes) {
+            const uint32_t r = (uint32_t)o;
+            o += align_up(bytes, 16);
+            return r;
+        };
+        s.mask = take((size_t)E * 8);
+        s.cnt = take((size_t)E * 4);
+        s.off = take(((size_t)E + 1) * 4);
+        s.gpre = take(((size_t)E + 1) * 4);
+        s.idx = take(P * 4);
+        s.w = take(P * 4);
+        s.perm = take(P * 4);
+        s.ipos = take(P * 4);
+        s.gexp = take((P + 64) * 4);
+        s.gpos = take((P + 64) * 4);
+        s.seg_c = take((P + (size_t)E + 70) * 8);
+        s.seg_i = take((P + (size_t)E + 70) * 4);
+        s.seg_cost = take((P + (size_t)E + 70) * 4);
+        s.tmp = take(32 * 8);
+        s.logit = take(T <= MT ? (size_t)T * E * 4 : 16);
+        s.ring_slots = layer_ring_slots(MT);
+        s.ring = take((size_t)(layer_threads(MT) / 32) * s.ring_slots * kSlotBytes);
+        off = o;
+    }
+    s.y_off = off;
+    off += out_rows ? align_up((size_t)rows_per_cta * (k + 1) * 4, 16) : 0;
+    s.bytes = off;
+    return s;
+}
+
+// ---------------------------------------------------------------------------
+// small block-level helpers (every thread of the block calls them)
+
+// Exclusive prefix sum of v[0..n) in place (int), returns the total.
+__device__ __forceinline__ int block_excl_scan(int* v, int n, int* tmp32)
+{
+    // each thread owns a contiguous run
+    const int nthr = blockDim.x, nwarp = nthr >> 5;
+    const int per = (n + nthr - 1) / nthr;
+    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+    int s = 0;
+    for (int i = lo; i < hi; ++i) s += v[i];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) tmp32[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarp ? tmp32[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < nwarp) tmp32[lane] = w;  // inclusive warp totals
+    }
+    __syncthreads();
+    int run = incl - s + (warp > 0 ? tmp32[warp - 1] : 0);
+    const int total = tmp32[nwarp - 1];
+    for (int i = lo; i < hi; ++i) {
+        const int x = v[i];
+        v[i] = run;
+        run += x;
+    }
+    __syncthreads();
+    return total;
+}
+
+// Segment lookup: the segment s with pre[s] <= x < pre[s + 1] (pre ascending, pre[0] = 0).
+__device__ __forceinline__ int seg_find(const int* pre, int nseg, long long x)
+{
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long long)pre[mid] <= x) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+}  // namespace coli
+
+namespace coli {
+
+// ---------------------------------------------------------------------------
+// top-k of one token from register-held scores
+
+// Top-k of one token by one warp; lane l holds the router scores of experts
+// e = l + 32 i in l[i] (E <= 32 kPer).  Same rule as the layer's other top-k:
+// key = order-preserving image of c = sigmoid(logit) + bias (NaN -> -inf,
+// -0 -> +0) then the complement of the index, so larger keys mean (c desc,
+// index asc) and keys are unique.  Each lane sorts its keys (carrying the
+// unbiased sigmoid along); k rounds take the warp maximum of the heads, the
+// owner pops its head and hands out its sigmoid.  Lane j < k returns expert
+// and weight routed_scale * s_j / sum s.
+template <int kPer>
+__device__ __forceinline__ void topk_regs(const float (&l)[kPer], int E, int k, const float* __restrict__ sel_bias,
+                                          float routed_scale, float top_p, int& my_e, float& my_w)
+{
+    const int lane = threadIdx.x & 31;
+    unsigned long long key[kPer];
+    float sg[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = 0ull;
+        sg[i] = 0.f;
+        if (e < E) {
+            const float s = 1.0f / (1.0f + expf(-l[i]));
+            const float ci = s + sel_bias[e];
+            const float c = (ci == ci) ? ci + 0.0f : -INFINITY;
+            const uint32_t u = __float_as_uint(c);
+            const uint32_t m = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+            key[i] = ((unsigned long long)m << 32) | (uint32_t)(0xFFFFu - e);
+            sg[i] = s;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kPer; ++r)
+#pragma unroll
+        for (int i = r & 1; i + 1 < kPer; i += 2) {
+            const bool sw = key[i] < key[i + 1];
+            const unsigned long long a = key[i], b = key[i + 1];
+            const float sa = sg[i], sb = sg[i + 1];
+            key[i] = sw ? b : a;
+            key[i + 1] = sw ? a : b;
+            sg[i] = sw ? sb : sa;
+            sg[i + 1] = sw ? sa : sb;
+        }
+    my_e = -1;
+    float my_s = 0.f;
+    for (int j = 0; j < k; ++j) {
+        unsigned long long best = key[0];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+            best = other > best ? other : best;
+        }
+        const int e = (int)(0xFFFFu - (uint32_t)(best & 0xFFFFu));
+        float popped = 0.f;
+        if (key[0] == best) {  // the unique owner (lane e % 32) pops its head
+            popped = sg[0];
+#pragma unroll
+            for (int i = 0; i + 1 < kPer; ++i) {
+                key[i] = key[i + 1];
+                sg[i] = sg[i + 1];
+            }
+            key[kPer - 1] = 0ull;
+            sg[kPer - 1] = 0.f;
+        }
+        const float s = __shfl_sync(0xFFFFFFFFu, popped, e & 31);
+        if (lane == j) {
+            my_e = e;
+            my_s = s;
+        }
+    }
+    topk_weights(k, top_p, routed_scale, my_e, my_s, my_w);
+}
+
+// Top-k of token t for more than 256 experts (same rule and result as
+// topk_regs), with few registers: k rounds of a warp arg-max over the scores,
+// re-read from global memory each round; taken experts are marked in a
+// per-lane bit mask (expert lane + 32 i <-> bit i).
+__device__ __noinline__ void topk_rounds_global(const float* __restrict__ part, int npc, int T, int t, int E, int k,
+                                                const float* __restrict__ sel_bias, float routed_scale, float top_p,
+                                                int& my_e, float& my_w)
+{
+    const int lane = threadIdx.x & 31;
+    unsigned int taken = 0u;
+    my_e = -1;
+    float my_s = 0.f;
+    for (int j = 0; j < k; ++j) {
+        unsigned long long best = 0ull;
+        float best_s = 0.f;
+        for (int i = 0; 32 * i < E; ++i) {
+            const int e = lane + 32 * i;
+            if (e >= E || ((taken >> i) & 1u)) continue;
+            float l = 0.f;
+            for (int p = 0; p < npc; ++p) l += part[((size_t)p * T + t) * E + e];
+            const float s = 1.0f / (1.0f + expf(-l));
+            const float ci = s + sel_bias[e];
+            const float c = (ci == ci) ? ci + 0.0f : -INFINITY;
+            const uint32_t uu = __float_as_uint(c);
+            const uint32_t m = (uu & 0x80000000u) ? ~uu : (uu | 0x80000000u);
+            const unsigned long long key = ((unsigned long long)m << 32) | (uint32_t)(0xFFFFu - e);
+            if (key > best) {
+                best = key;
+                best_s = s;
+            }
+        }
+        unsigned long long w = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, w, o);
+            w = other > w ? other : w;
+        }
+        const int e = (int)(0xFFFFu - (uint32_t)(w & 0xFFFFu));
+        const float s = __shfl_sync(0xFFFFFFFFu, best_s, e & 31);
+        if (lane == (e & 31)) taken |= 1u << (e >> 5);
+        if (lane == j) {
+            my_e = e;
+            my_s = s;
+        }
+    }
+    topk_weights(k, top_p, routed_scale, my_e, my_s, my_w);
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+
+// 64-bit exclusive prefix sum of v[0..n) in place; returns the total.
+__device__ __forceinline__ long long block_excl_scan64(long long* v, int n, long long* tmp32)
+{
+    const int nthr = blockDim.x, nwarp = nthr >> 5;
+    const int per = (n + nthr - 1) / nthr;
+    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+    long long s = 0;
+    for (int i = lo; i < hi; ++i) s += v[i];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) tmp32[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        long long w = lane < nwarp ? tmp32[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < nwarp) tmp32[lane] = w;
+    }
+    __syncthreads();
+    long long run = incl - s + (warp > 0 ? tmp32[warp - 1] : 0);
+    const long long total = tmp32[nwarp - 1];
+    for (int i = lo; i < hi; ++i) {
+        const long long x = v[i];
+        v[i] = run;
+        run += x;
+    }
+    __syncthreads();
+    return total;
+}
+
+// Work-list segments of one phase: segment s holds n items of cost c each.
+// After seg_prepare, ipre[s] / cpre[s] are the item / cost offsets of segment s
+// (ipre[nseg], cpre[nseg] the totals).
+struct SegTable {
+    int* ipre;        // [nseg + 1]
+    long long* cpre;  // [nseg + 1]
+    int* cost;        // [nseg]
+    long long* tmp;   // [32]
+    int nseg;
+};
+
+// Largest s in [0, n] with a[s] <= x (a ascending, a[0] <= x).
+template <typename V>
+__device__ __forceinline__ int last_le(const V* a, int n, long long x)
+{
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long long)a[mid] <= x) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// This CTA's items of the phase: those whose start cost lies in
+// [C b / G, C (b + 1) / G).
+__device__ __forceinline__ void seg_cta_range(const SegTable& st, int& lo, int& hi)
+{
+    const long long C = st.cpre[st.nseg];
+    auto first = [&](long long x) -> int {
+        const int s = last_le(st.cpre, st.nseg, x);
+        if (s >= st.nseg) return st.ipre[st.nseg];
+        const long long c = st.cost[s] > 0 ? st.cost[s] : 1;
+        const long long r = (x - st.cpre[s] + c - 1) / c;
+        const long long n = st.ipre[s + 1] - st.ipre[s];
+        return st.ipre[s] + (int)(r < n ? r : n);
+    };
+    lo = first(C * (long long)blockIdx.x / gridDim.x);
+    hi = first(C * (long long)(blockIdx.x + 1) / gridDim.x);
+}
+
+// Union tables in shared memory (every CTA computes the same ones).
+struct UnionSmem {
+    unsigned long long* mask;  // [E] tokens that chose expert e
+    int* cnt;                  // [E]
+    int* off;                  // [E + 1] first sorted position of expert e
+    int* gpre;                 // [E + 1] first group of expert e
+    int* idx;                  // [P] routing (token-major)
+    float* w;                  // [P]
+    int* perm;                 // [P] pair id at each sorted position
+    int* ipos;                 // [P] sorted position of each pair
+    int* gexp;                 // [P + 64] expert of each routed group
+    int* gpos;                 // [P + 64] first sorted position of each routed group
+    int* seg_i;                // segment table storage
+    long long* seg_c;
+    int* seg_cost;
+    long long* tmp;            // [32]
+};
+
+__device__ __forceinline__ UnionSmem union_smem(unsigned char* base, const LayerSmem& ls)
+{
+    UnionSmem u;
+    u.mask = reinterpret_cast<unsigned long long*>(base + ls.mask);
+    u.cnt = reinterpret_cast<int*>(base + ls.cnt);
+    u.off = reinterpret_cast<int*>(base + ls.off);
+    u.gpre = reinterpret_cast<int*>(base + ls.gpre);
+    u.idx = reinterpret_cast<int*>(base + ls.idx);
+    u.w = reinterpret_cast<float*>(base + ls.w);
+    u.perm = reinterpret_cast<int*>(base + ls.perm);
+    u.ipos = reinterpret_cast<int*>(base + ls.ipos);
+    u.gexp = reinterpret_cast<int*>(base + ls.gexp);
+    u.gpos = reinterpret_cast<int*>(base + ls.gpos);
+    u.seg_c = reinterpret_cast<long long*>(base + ls.seg_c);
+    u.seg_i = reinterpret_cast<int*>(base + ls.seg_i);
+    u.seg_cost = reinterpret_cast<int*>(base + ls.seg_cost);
+    u.tmp = reinterpret_cast<long long*>(base + ls.tmp);
+    return u;
+}
+
+
+// Prefix sums of a segment table whose counts are in ipre[0..n) and per-item
+// costs in cost[0..n) (all threads call this).
+__device__ __forceinline__ SegTable seg_prepare(const UnionSmem& u, int nseg)
+{
+    SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
+    for (int s = threadIdx.x; s < nseg; s += blockDim.x) st.cpre[s] = (long long)st.ipre[s] * st.cost[s];
+    if (threadIdx.x == 0) {
+        st.ipre[nseg] = 0;
+        st.cpre[nseg] = 0;
+    }
+    __syncthreads();
+    block_excl_scan(st.ipre, nseg + 1, reinterpret_cast<int*>(u.tmp));
+    block_excl_scan64(st.cpre, nseg + 1, u.tmp);
+    return st;
+}
+
+}  // namespace coli
+
+namespace coli {
+
+// Grid-barrier word of this cooperative launch (nullptr if the launch was not cooperative).
+__device__ __forceinline__ unsigned int* launch_barrier_word()
+{
+    cooperative_groups::details::grid_workspace* ws = cooperative_groups::details::get_grid_workspace();
+    return ws ? &ws->barrier : nullptr;
+}
+
+// Partial router scores of one piece: chunks c = lane + 32 p of router row e
+// (32 fp32 weights each) against the nt staged activation vectors; the warp's
+// sums go to logit_part[p][t][e].
+template <int NT>
+__device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, int nt, const StageGeom& g,
+                                             const float4* xs)
+{
+    const int lane = threadIdx.x & 31;
+    const int c = lane + 32 * p;
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+    if (c < g.nch) {
+        const float4* wrow = reinterpret_cast<const float4*>(a.w_router + (size_t)e * a.H) + (size_t)c * 8;
+        float4 wv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) wv[j] = __ldg(wrow + j);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            if (t < nt) {
+                const float4* xr = xs + (size_t)t * g.f4 + p * 256;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 xv = xr[j * 32 + (lane ^ j)];  // swapped pairs (x1, x0, x3, x2)
+                    acc[t] = fmaf(wv[j].x, xv.y, acc[t]);
+                    acc[t] = fmaf(wv[j].y, xv.x, acc[t]);
+                    acc[t] = fmaf(wv[j].z, xv.w, acc[t]);
+                    acc[t] = fmaf(wv[j].w, xv.z, acc[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        if (t < nt) {
+            const float v = warp_sum(acc[t]);
+            if (lane == 0) a.logit_part[((size_t)p * a.T + t) * a.E + e] = v;
+        }
+    }
+}
+
+// Cost per item of a row-pair item of m vectors: bytes of the two rows (in
+// 256-byte units) times (3 + m) / 4, the int4 decode being shared by the
+// vectors and the multiply-adds not.
+__device__ __forceinline__ int pair_cost(int K, int m) { return max(1, (K + K / 8) / 256) * (3 + m); }
+
+// The layer, T <= 64 tokens.  MT = tokens per group (vectors per item);
+// kOutRows: one token, down and combine by output rows.
+template <int MT, bool kBf16, bool kOutBf16, bool kOutRows>
+__global__ void __launch_bounds__(layer_threads(MT), 1)
+moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
+{
+    constexpr int kLayerThreads = layer_threads(MT);
+    constexpr int kLayerWarps = kLayerThreads / 32;
+    extern __shared__ __align__(16) unsigned char lsm[];
+    constexpr int P_GU = layer_ring_slots(MT);  // ring slots (steps in flight + 1) of the streams
+    constexpr int P_DN = layer_ring_slots(MT);
+    const int H = a.H, F = a.F, E = a.E, k = a.k, T = a.T;
+    const int P = T * k;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const StageGeom gH = stage_geom(H), gF = stage_geom(F);
+    float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
+    float* xcorr = reinterpret_cast<float*>(lsm + ls.x_off + (size_t)ls.nx * gH.f4 * 16);
+    float4* hs = reinterpret_cast<float4*>(lsm + ls.h_off);
+    float* hcorr = reinterpret_cast<float*>(lsm + ls.h_off + (size_t)ls.nh * gF.f4 * 16);
+    const UnionSmem u = union_smem(lsm, ls);
+    float* ypart = reinterpret_cast<float*>(lsm + ls.y_off);
+    unsigned char* ring = lsm + ls.ring + (size_t)(threadIdx.x >> 5) * P_GU * kSlotBytes;  // this warp's ring
+
+    unsigned int* bar = launch_barrier_word();
+    if (!bar) {  // not a cooperative launch: nothing can be synchronised (same answer in every CTA)
+        if (blockIdx.x == 0 && threadIdx.x == 0) *a.err = 3;
+        return;
+    }
+    const unsigned long long deadline = layer_ns() + a.wait_ns;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *a.err = 0;
+    stamp(a, 0);
+    const bool all_x = T <= MT;  // every token's activations staged once for the whole call
+    const int n_sg = (T + MT - 1) / MT;  // shared-expert groups
+
+    auto stage_x = [&](int n, auto token_of) {
+        stage_vectors<kBf16>(a.x, H, n, token_of, gH, xs, xcorr);
+    };
+    auto stage_h = [&](int n, auto pos_of) {
+        stage_vectors<false>(a.h, F, n, pos_of, gF, hs, hcorr);
+    };
+
+    // gate/up item finisher: h[pos_t, n] = silu(gate) * up for the group's vectors
+    auto gateup_finish = [&](int n, int pos0, bool, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            if (t < v.m) {
+                const float gv = warp_sum(tot[0][t]);
+                const float uv = warp_sum(tot[1][t]);
+                const int pos = pos0 + t;
+                if (lane == 0 && COLI_IN_BOUNDS(pos >= 0 && pos < P + T && n >= 0 && n < F, a.err))
+                    a.h[(size_t)pos * F + n] = gv / (1.0f + expf(-gv)) * uv;
+            }
+        }
+    };
+
+    // ======================= phase A: router pieces, shared gate/up =======================
+    {
+        // Router pieces (scored here up to 4 tokens): block b takes pieces b, b + G, ... and its
+        // warps one each, so every block has about the same number.  The shared expert's gate/up
+        // rows are cut into equal-cost ranges.  The first gate/up loads are issued before the
+        // activations are staged and before the warp's router piece is computed (engine hook).
+        const int nrp = a.n_pieces == 0 ? gH.per_lane : 0;  // router pieces per row (computed here)
+        auto router_pieces = [&]() {
+            const int total = E * nrp;
+            for (int i = blockIdx.x + gridDim.x * warp; i < total; i += gridDim.x * kLayerWarps)
+                router_piece<MT>(a, i / nrp, i % nrp, T, gH, xs);
+        };
+        auto stage_all = [&]() {
+            stage_x(T, [](int t) { return t; });
+            __syncthreads();
+            stamp(a, 1);
+        };
+        const int nseg = n_sg;
+        for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
+            u.seg_i[s] = F;
+            u.seg_cost[s] = pair_cost(H, min(MT, T - s * MT));
+        }
+        __syncthreads();
+        const SegTable st = seg_prepare(u, nseg);
+        int lo, hi;
+        seg_cta_range(st, lo, hi);
+        bool ran = false;
+        for (int s = 0; s < nseg; ++s) {
+            const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
+            if (s_lo >= s_hi) continue;
+            const int t0 = s * MT, m = min(MT, T - t0);
+            const int base = st.ipre[s];
+            auto rows_of = [&](int j, RowPair& r) {
+                const size_t row = (size_t)E * F + (j - base);
+                r.q0 = a.gate_q + row * (H / 2);
+                r.q1 = a.up_q + row * (H / 2);
+                r.s0 = a.gate_s + row * (H / kGroup);
+                r.s1 = a.up_s + row * (H / kGroup);
+            };
+            auto vecs_of = [&](int, VecSet<MT>& v) {
+                v.m = m;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    const int vi = all_x ? t0 + t : t;
+                    v.x4[t] = vi * gH.f4;
+                    v.cr[t] = vi * gH.nch;
+                }
+            };
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+                gateup_finish(j - base, P + t0, true, v, tot);
+            };
+            auto hook = [&]() {
+                if (all_x) {
+                    if (!ran) {
+                        stage_all();
+                        router_pieces();
+                    }
+                } else {  // this group's tokens (the router ran before the launch)
+                    __syncthreads();
+                    stage_x(m, [t0](int t) { return t0 + t; });
+                    __syncthreads();
+                }
+            };
+            const int first = s_lo + warp;
+            const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
+            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
+                                       fin, hook);
+            ran = true;
+        }
+        if (!ran && all_x) {  // no gate/up rows in this block: activations and router pieces only
+            stage_all();
+            router_pieces();
+        }
+    }
+    stamp(a, 2);
+    grid_barrier(bar, deadline, a.err);
+    stamp(a, 3);
+
+    // ======================= phase B: top-k, union, routed gate/up =======================
+    const int S1 = k + 1;  // one token: slots (routed in order, shared last)
+    const int pr_lo = (int)((long long)(H / 2) * blockIdx.x / gridDim.x);  // one token: this CTA's output row pairs
+    const int npr = (int)((long long)(H / 2) * (blockIdx.x + 1) / gridDim.x) - pr_lo;
+    float* s_logit = reinterpret_cast<float*>(lsm + ls.logit);
+    const int npc = a.n_pieces == 0 ? gH.per_lane : a.n_pieces;
+    // router scores of the tokens: sums of the per-piece partials (independent loads), into shared memory
+    auto sum_pieces = [&]() {
+        for (int i = threadIdx.x; i < T * E; i += kLayerThreads) {
+            float v = 0.f;
+#pragma unroll
+            for (int p = 0; p < 16; ++p)
+                if (p < npc) v += a.logit_part[(size_t)p * T * E + i];
+            s_logit[i] = v;
+        }
+        __syncthreads();
+    };
+    if constexpr (kOutRows) {
+        sum_pieces();
+        if (warp == 0) {
+            // the token's top-k, then the union of its k experts: ascending expert order
+            int my_e;
+            float my_w;
+            if (E <= 256) {
+                float l[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int e = lane + 32 * i;
+                    l[i] = e < E ? s_logit[e] : 0.f;
+                }
+                topk_regs<8>(l, E, k, a.sel_bias, a.routed_scale, a.top_p, my_e, my_w);
+            } else {
+                topk_rounds_global(a.logit_part, npc, 1, 0, E, k, a.sel_bias, a.routed_scale, a.top_p, my_e, my_w);
+            }
+            // kept experts (top-p may drop slots: expert -1) in ascending order
+            int rank = 0;
+            for (int i = 0; i < k; ++i) {
+                const int ei = __shfl_sync(0xFFFFFFFFu, my_e, i);
+                rank += (ei >= 0 && ei < my_e) ? 1 : 0;
+            }
+            const int n_kept = __popc(__ballot_sync(0xFFFFFFFFu, lane < k && my_e >= 0));
+            if (lane < k) {
+                u.idx[lane] = my_e;
+                u.w[lane] = my_w;
+                u.ipos[lane] = my_e >= 0 ? rank : -1;
+                if (my_e >= 0) {
+                    u.perm[rank] = lane;
+                    u.gexp[rank] = my_e;
+                    u.gpos[rank] = rank;
+                }
+                if (blockIdx.x == 0) {
+                    a.idx_out[lane] = my_e;
+                    a.w_out[lane] = my_w;
+                }
+            }
+            if (lane == 0) reinterpret_cast<int*>(u.tmp)[0] = n_kept;
+        } else {
+            // meanwhile: the shared expert's h, and its down rows for this CTA's output rows
+            const int tid = threadIdx.x - 32, nthr = kLayerThreads - 32;
+            stage_vectors<false>(a.h, F, 1, [&](int) { return P; }, gF, hs + (size_t)k * gF.f4, hcorr + (size_t)k * gF.nch,
+                                 tid, nthr);
+            asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+            auto rows_of = [&](int j, RowPair& r) {
+                const size_t row = (size_t)E * H + 2 * (pr_lo + j);
+                r.q0 = a.down_q + row * (F / 2);
+                r.q1 = r.q0 + F / 2;
+                r.s0 = a.down_s + row * (F / kGroup);
+                r.s1 = r.s0 + F / kGroup;
+            };
+            auto vecs_of = [&](int, VecSet<MT>& v) {
+                v.m = 1;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    v.x4[t] = k * gF.f4;
+                    v.cr[t] = k * gF.nch;
+                }
+            };
+            auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
+                const float y0 = warp_sum(tot[0][0]), y1 = warp_sum(tot[1][0]);
+                if (lane == 0) {
+                    ypart[(2 * j) * S1 + k] = y0;
+                    ypart[(2 * j + 1) * S1 + k] = y1;
+                }
+            };
+            const int first = warp - 1, nw = kLayerWarps - 1;
+            const int nj = first < npr ? (npr - first + nw - 1) / nw : 0;
+            stream_row_pairs<MT, P_DN>(first, nw, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin);
+        }
+        __syncthreads();
+        stamp(a, 4);
+        // routed gate/up: the kept experts x F rows, equal cost, an even split
+        const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
+        const int total = n_kept * F;
+        const int lo = (int)((long long)total * blockIdx.x / gridDim.x);
+        const int hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
+        auto rows_of = [&](int j, RowPair& r) {
+            const int g = j / F;
+            int e = u.gexp[g];
+            if (!COLI_IN_BOUNDS(e >= 0 && e < E, a.err)) e = 0;
+            const size_t row = (size_t)e * F + (j - g * F);
+            r.q0 = a.gate_q + row * (H / 2);
+            r.q1 = a.up_q + row * (H / 2);
+            r.s0 = a.gate_s + row * (H / kGroup);
+            r.s1 = a.up_s + row * (H / kGroup);
+        };
+        auto vecs_of = [&](int, VecSet<MT>& v) {
+            v.m = 1;
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                v.x4[t] = 0;
+                v.cr[t] = 0;
+            }
+        };
+        auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+            const int g = j / F;
+            gateup_finish(j - g * F, g, false, v, tot);
+        };
+        const int first = lo + warp;
+        const int nj = first < hi ? (hi - first + kLayerWarps - 1) / kLayerWarps : 0;
+        stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of, fin);
+    } else {
+        const bool scored_here = all_x;  // the kernel scored the tokens (pieces summed into shared memory)
+        if (scored_here) sum_pieces();
+        for (int t = warp; t < T; t += kLayerWarps) {
+            int my_e;
+            float my_w;
+            if (E <= 256) {
+                float l[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int e = lane + 32 * i;
+                    l[i] = e >= E ? 0.f : scored_here ? s_logit[t * E + e] : a.logit_part[(size_t)t * E + e];
+                }
+                topk_regs<8>(l, E, k, a.sel_bias, a.routed_scale, a.top_p, my_e, my_w);
+            } else {
+                topk_rounds_global(a.logit_part, npc, T, t, E, k, a.sel_bias, a.routed_scale, a.top_p, my_e, my_w);
+            }
+            if (lane < k) {
+                u.idx[t * k + lane] = my_e;
+                u.w[t * k + lane] = my_w;
+                if (blockIdx.x == 0) {
+                    a.idx_out[t * k + lane] = my_e;
+                    a.w_out[t * k + lane] = my_w;
+                }
+            }
+        }
+        for (int e = threadIdx.x; e < E; e += kLayerThreads) u.mask[e] = 0ull;
+        __syncthreads();
+        // union: token masks per expert, counts, offsets, stable positions
+        for (int p = threadIdx.x; p < P; p += kLayerThreads)
+            if (u.idx[p] >= 0 && COLI_IN_BOUNDS(u.idx[p] < E, a.err))  // dropped slots (-1) have no expert
+                atomicOr(&u.mask[u.idx[p]], 1ull << (p / k));
+        __syncthreads();
+        for (int e = threadIdx.x; e <= E; e += kLayerThreads) {
+            const int c = e < E ? __popcll(u.mask[e]) : 0;
+            u.off[e] = c;
+            u.gpre[e] = (c + MT - 1) / MT;
+            if (e < E) u.cnt[e] = c;
+        }
+        __syncthreads();
+        block_excl_scan(u.off, E + 1, reinterpret_cast<int*>(u.tmp));
+        const int n_rg = block_excl_scan(u.gpre, E + 1, reinterpret_cast<int*>(u.tmp));
+        for (int p = threadIdx.x; p < P; p += kLayerThreads) {
+            const int t = p / k, e = u.idx[p];
+            if (e < 0) {
+                u.ipos[p] = -1;
+                continue;
+            }
+            const unsigned long long below = t == 0 ? 0ull : (u.mask[e] & ((1ull << t) - 1ull));
+            const int pos = u.off[e] + __popcll(below);
+            if (!COLI_IN_BOUNDS(e < E && pos < P, a.err)) {
+                u.ipos[p] = -1;
+                continue;
+            }
+            u.perm[pos] = p;
+            u.ipos[p] = pos;
+        }
+        for (int e = threadIdx.x; e < E; e += kLayerThreads) {
+            const int c = u.cnt[e];
+            for (int i = 0, g = u.gpre[e]; i * MT < c; ++i, ++g) {
+                u.gexp[g] = e;
+                u.gpos[g] = u.off[e] + i * MT;
+            }
+        }
+        __syncthreads();
+
+        // segments: [shared down groups (several tokens)] + routed gate/up groups
+        const int n_sd = kOutRows ? 0 : n_sg;
+        const int nseg = n_sd + n_rg;
+        for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
+            if (s < n_sd) {
+                const int m = min(MT, T - s * MT);
+                u.seg_i[s] = H / 2;
+                u.seg_cost[s] = pair_cost(F, m);
+            } else {
+                const int g = s - n_sd, e = u.gexp[g];
+                const int m = min(MT, u.off[e] + u.cnt[e] - u.gpos[g]);
+                u.seg_i[s] = F;
+                u.seg_cost[s] = pair_cost(H, m);
+            }
+        }
+        __syncthreads();
+        const SegTable st = seg_prepare(u, nseg);
+        int lo, hi;
+        seg_cta_range(st, lo, hi);
+
+        // shared expert's down rows (several tokens), one run per shared group
+        for (int s = 0; s < n_sd; ++s) {
+            const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
+            if (s_lo >= s_hi) continue;
+            const int t0 = s * MT, m = min(MT, T - t0);
+            __syncthreads();
+            stage_h(m, [&](int t) { return P + t0 + t; });
+            __syncthreads();
+            const int base = st.ipre[s];
+            auto rows_of = [&](int j, RowPair& r) {
+                const size_t row = (size_t)E * H + 2 * (j - base);
+                r.q0 = a.down_q + row * (F / 2);
+                r.q1 = r.q0 + F / 2;
+                r.s0 = a.down_s + row * (F / kGroup);
+                r.s1 = r.s0 + F / kGroup;
+            };
+            auto vecs_of = [&](int, VecSet<MT>& v) {
+                v.m = m;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    v.x4[t] = t * gF.f4;
+                    v.cr[t] = t * gF.nch;
+                }
+            };
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+                const int n = 2 * (j - base);
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    if (t < v.m) {
+                        const float y0 = warp_sum(tot[0][t]), y1 = warp_sum(tot[1][t]);
+                        if (lane == 0) {
+                            float* yr = a.y + (size_t)(P + t0 + t) * H + n;
+                            yr[0] = y0;
+                            yr[1] = y1;
+                        }
+                    }
+                }
+            };
+            const int first = s_lo + warp;
+            const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
+            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin);
+        }
+
+        // routed gate/up: one run over all routed groups when every token is staged,
+        // else one run per group (its tokens staged)
+        const int r_lo = max(lo, st.ipre[n_sd]), r_hi = hi;
+        for (int s = n_sd; s < nseg && r_lo < r_hi; ++s) {
+            int s_lo, s_hi;
+            if (all_x) {
+                if (s != n_sd) break;
+                s_lo = r_lo;
+                s_hi = r_hi;
+            } else {
+                s_lo = max(r_lo, st.ipre[s]);
+                s_hi = min(r_hi, st.ipre[s + 1]);
+                if (s_lo >= s_hi) continue;
+                const int g = s - n_sd, e = u.gexp[g], p0 = u.gpos[g];
+                const int m = min(MT, u.off[e] + u.cnt[e] - p0);
+                __syncthreads();
+                stage_x(m, [&](int t) { return u.perm[p0 + t] / k; });
+                __syncthreads();
+            }
+            auto seg_of = [&](int j) { return all_x ? last_le(st.ipre, nseg - 1, j) : s; };
+            auto rows_of = [&](int j, RowPair& r) {
+                const int sj = seg_of(j);
+                int e = u.gexp[sj - n_sd];
+                if (!COLI_IN_BOUNDS(e >= 0 && e < E && j - st.ipre[sj] < F, a.err)) e = 0;
+                const size_t row = (size_t)e * F + (j - st.ipre[sj]);
+                r.q0 = a.gate_q + row * (H / 2);
+                r.q1 = a.up_q + row * (H / 2);
+                r.s0 = a.gate_s + row * (H / kGroup);
+                r.s1 = a.up_s + row * (H / kGroup);
+            };
+            auto vecs_of = [&](int j, VecSet<MT>& v) {
+                const int g = seg_of(j) - n_sd, e = u.gexp[g], p0 = u.gpos[g];
+                v.m = min(MT, u.off[e] + u.cnt[e] - p0);
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    const int vi = all_x ? (t < v.m ? u.perm[p0 + t] / k : 0) : t;
+                    v.x4[t] = vi * gH.f4;
+                    v.cr[t] = vi * gH.nch;
+                }
+            };
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+                const int sj = seg_of(j);
+                gateup_finish(j - st.ipre[sj], u.gpos[sj - n_sd], false, v, tot);
+            };
+            const int first = s_lo + warp;
+            const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
+            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of, fin);
+        }
+    }
+    stamp(a, 5);
+    if constexpr (!kOutRows) grid_barrier(bar, deadline, a.err);
+
+    // ======================= phase C: down =======================
+    if constexpr (kOutRows) {
+        // one token: this CTA's output row pairs of the k routed slots; the loads of
+        // the first rows are issued before the grid barrier (the weights do not
+        // depend on it), the routed h vectors are staged after it
+        const int S = S1;
+        // item j = (group g = j / npr: the g-th kept expert in ascending order, row pair)
+        const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
+        auto rows_of = [&](int j, RowPair& r) {
+            const int slot = j / npr, pr = pr_lo + (j - slot * npr);
+            int e = u.gexp[slot];
+            if (!COLI_IN_BOUNDS(e >= 0 && e < E && 2 * pr + 1 < H, a.err)) e = 0;
+            const size_t row = (size_t)e * H + 2 * pr;
+            r.q0 = a.down_q + row * (F / 2);
+            r.q1 = r.q0 + F / 2;
+            r.s0 = a.down_s + row * (F / kGroup);
+            r.s1 = r.s0 + F / kGroup;
+        };
+        auto vecs_of = [&](int j, VecSet<MT>& v) {
+            const int slot = j / npr;
+            v.m = 1;
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                v.x4[t] = slot * gF.f4;
+                v.cr[t] = slot * gF.nch;
+            }
+        };
+        auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
+            const int slot = j / npr, pl = j - slot * npr;
+            const float y0 = warp_sum(tot[0][0]), y1 = warp_sum(tot[1][0]);
+            if (lane == 0) {
+                ypart[(2 * pl) * S + slot] = y0;
+                ypart[(2 * pl + 1) * S + slot] = y1;
+            }
+        };
+        auto hook = [&]() {
+            grid_barrier(bar, deadline, a.err);
+            stamp(a, 6);
+            stage_h(n_kept, [&](int g) { return g; });  // h of the g-th kept expert sits at position g
+            __syncthreads();
+            stamp(a, 7);
+        };
+        const int total = npr * n_kept;
+        const int first = warp;
+        const int nj = first < total ? (total - first + kLayerWarps - 1) / kLayerWarps : 0;
+        stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin,
+                                   hook);
+        __syncthreads();
+        stamp(a, 8);
+        for (int i = threadIdx.x; i < 2 * npr; i += kLayerThreads) {
+            float acc = 0.f;
+            for (int j = 0; j < k; ++j)
+                if (u.ipos[j] >= 0) acc = fmaf(u.w[j], ypart[i * S + u.ipos[j]], acc);
+            acc += ypart[i * S + k];
+            const int n = 2 * pr_lo + i;
+            if constexpr (kOutBf16) static_cast<uint16_t*>(a.out)[n] = float_to_bf16_bits(acc);
+            else static_cast<float*>(a.out)[n] = acc;
+        }
+    } else {
+        // several tokens: routed down rows, one partial output row per pair (routing weight applied)
+        const int n_rg = u.gpre[E];
+        const int nseg = n_rg;
+        for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
+            const int e = u.gexp[s];
+            const int m = min(MT, u.off[e] + u.cnt[e] - u.gpos[s]);
+            u.seg_i[s] = H / 2;
+            u.seg_cost[s] = pair_cost(F, m);
+        }
+        __syncthreads();
+        const SegTable st = seg_prepare(u, nseg);
+        int lo, hi;
+        seg_cta_range(st, lo, hi);
+        for (int s = 0; s < nseg; ++s) {
+            const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
+            if (s_lo >= s_hi) continue;
+            const int e = u.gexp[s], p0 = u.gpos[s];
+            const int m = min(MT, u.off[e] + u.cnt[e] - p0);
+            __syncthreads();
+            stage_h(m, [&](int t) { return p0 + t; });
+            __syncthreads();
+            const int base = st.ipre[s];
+            auto rows_of = [&](int j, RowPair& r) {
+                const size_t row = (size_t)e * H + 2 * (j - base);
+                r.q0 = a.down_q + row * (F / 2);
+                r.q1 = r.q0 + F / 2;
+                r.s0 = a.down_s + row * (F / kGroup);
+                r.s1 = r.s0 + F / kGroup;
+            };
+            auto vecs_of = [&](int, VecSet<MT>& v) {
+                v.m = m;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    v.x4[t] = t * gF.f4;
+                    v.cr[t] = t * gF.nch;
+                }
+            };
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+                const int n = 2 * (j - base);
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    if (t < v.m) {
+                        const float y0 = warp_sum(tot[0][t]), y1 = warp_sum(tot[1][t]);
+                        if (lane == 0 && COLI_IN_BOUNDS(p0 + t < P && n + 1 < H, a.err)) {
+                            const float wt = u.w[u.perm[p0 + t]];
+                            float* yr = a.y + (size_t)(p0 + t) * H + n;
+                            yr[0] = wt * y0;
+                            yr[1] = wt * y1;
+                        }
+                    }
+                }
+            };
+            const int first = s_lo + warp;
+            const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
+            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin);
+        }
+        grid_barrier(bar, deadline, a.err);
+
+        // ======================= phase D: combine =======================
+        const int per_row = H / 4;
+        const int total = T * per_row;
+        const int stride = gridDim.x * kLayerThreads;
+        for (int i = blockIdx.x * kLayerThreads + threadIdx.x; i < total; i += stride) {
+            const int t = i / per_row, n = (i - t * per_row) * 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j <= k; ++j) {
+                const int pos = j < k ? u.ipos[t * k + j] : P + t;
+                if (pos < 0) continue;  // a slot dropped by top-p
+                if (!COLI_IN_BOUNDS(pos < P + T, a.err)) continue;
+                const float4 v = *reinterpret_cast<const float4*>(a.y + (size_t)pos * H + n);
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            if constexpr (kOutBf16) {
+                uint2 o;
+                o.x = (uint32_t)float_to_bf16_bits(acc.x) | ((uint32_t)float_to_bf16_bits(acc.y) << 16);
+                o.y = (uint32_t)float_to_bf16_bits(acc.z) | ((uint32_t)float_to_bf16_bits(acc.w) << 16);
+                *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + (size_t)t * H + n) = o;
+            } else {
+                *reinterpret_cast<float4*>(static_cast<float*>(a.out) + (size_t)t * H + n) = acc;
+            }
+        }
+    }
+    stamp(a, 9);
+}
+
+}  // namespace coli

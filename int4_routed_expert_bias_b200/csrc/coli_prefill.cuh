@@ -75,7 +75,6 @@ static_assert(kPfBStageBytes % 1024 == 0 && kPfRawStageBytes % 1024 == 0, "swizz
 // ---------------------------------------------------------------------------
 // PTX wrappers
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 __device__ __forceinline__ unsigned long long global_ns()
 {
@@ -306,6 +305,7 @@ struct PrefillArgs {
     uint16_t* h;              // gate/up out: bf16 [P + T, F], permuted rows
     uint16_t* ys;             // down out: bf16 [T, k + 1, H]
     int* err;
+    unsigned long long wait_ns;  // limit of every pipeline wait (teardown drains keep their own)
 };
 
 // tq0 / tq1: int4 bytes of tile rows 0-63 / 64-127 (box 128 B x 64 rows, 128-byte
@@ -360,7 +360,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap tq0, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
-    const unsigned long long deadline = global_ns() + kPfWaitNs;
+    const unsigned long long deadline = global_ns() + a.wait_ns;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -471,7 +471,10 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap tq0, const __grid_consta
                         t = pos - a.P;
                         slot = a.k;
                     }
-                    s_dst[c] = t * (a.k + 1) + slot;
+                    // destination row of ys [T, k+1, H]; the bounds-checked build parks a bad one on row 0
+                    const int dst = t * (a.k + 1) + slot;
+                    s_dst[c] = COLI_IN_BOUNDS(t >= 0 && slot >= 0 && slot <= a.k && (pos >= a.P || t < a.P / a.k),
+                                              a.err) ? dst : 0;
                     s_w[c] = a.pair_w[pos];
                 }
             }
@@ -588,13 +591,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap tq0, const __grid_consta
 // xg[pos, 8g + p] = x[pair_token[pos], 8g + sigma(p)].
 template <bool kXBf16>
 __global__ void prefill_gather_kernel(const void* __restrict__ x, const int32_t* __restrict__ pair_token, int Q,
-                                      int H, uint16_t* __restrict__ xg)
+                                      int T, int H, uint16_t* __restrict__ xg)
 {
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int g8 = H / 8;
     if (i >= (size_t)Q * g8) return;
     const int pos = (int)(i / g8), g = (int)(i - (size_t)pos * g8);
-    const int t = pair_token[pos];
+    int t = pair_token[pos];
+    if (!COLI_IN_BOUNDS(t >= 0 && t < T, nullptr)) t = 0;
     float v[8];
     if constexpr (kXBf16) {
         const uint4 r = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)t * H + 8 * g);
@@ -617,14 +621,17 @@ __global__ void prefill_gather_kernel(const void* __restrict__ x, const int32_t*
 }
 
 // out[t, n] = sum over slots j (routed in slot order, shared last) of ys[t, j, n].
+// Slots whose routing index is -1 (dropped by adaptive top-p) were never written and are skipped.
 template <bool kOutBf16>
-__global__ void slot_reduce_kernel(const uint16_t* __restrict__ ys, int T, int S, int H, void* __restrict__ out)
+__global__ void slot_reduce_kernel(const uint16_t* __restrict__ ys, int T, int S, int H,
+                                   const int32_t* __restrict__ topk_idx, void* __restrict__ out)
 {
     const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;  // 8 outputs per thread
     if (i >= (size_t)T * H) return;
     const size_t t = i / H, n = i - t * H;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < S; ++j) {
+        if (j < S - 1 && topk_idx[t * (S - 1) + j] < 0) continue;
         const uint4 v = *reinterpret_cast<const uint4*>(ys + ((size_t)t * S + j) * H + n);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll

@@ -79,51 +79,121 @@ router_logits_kernel(const void* __restrict__ x, int T, int H, const float* __re
     }
 }
 
-// logits[t, e] for large batches: a 64-token x 64-expert tile per block,
-// K-steps of 32 staged in shared memory, 4 x 4 outputs per thread, fp32.
-constexpr int kRtTile = 64;
-constexpr int kRtK = 32;
+// logits[t, e] for large batches: a 128-token x 64-expert tile per block of
+// 256 threads, 8 tokens x 4 experts per thread (packed fp32x2 multiply-adds
+// over expert pairs), K-steps of 16 staged in shared memory transposed to
+// [k][row] and double-buffered: the next step's global loads are in registers
+// while the current step is multiplied.  fp32 throughout; every output is one
+// sequential sum over k, as in the oracle's definition up to rounding order.
+constexpr int kRtT = 128, kRtE = 64, kRtK = 16;
+constexpr int kRtThreads = 256;
 
 template <bool kBf16>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kRtThreads)
 router_logits_tiled_kernel(const void* __restrict__ x, int T, int H, const float* __restrict__ w_router, int E,
                            float* __restrict__ logits)
 {
-    __shared__ float xs[kRtK][kRtTile + 4];
-    __shared__ float ws[kRtK][kRtTile + 4];
-    const int t0 = blockIdx.x * kRtTile, e0 = blockIdx.y * kRtTile;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // outputs (t0 + ty*4 + i, e0 + tx*4 + j)
-    float acc[4][4] = {};
-    for (int k0 = 0; k0 < H; k0 += kRtK) {
-        // stage 64 x 32 of x and of w_router, transposed to [k][row]
-        for (int i = threadIdx.x; i < kRtTile * kRtK / 4; i += 256) {
-            const int r = i / (kRtK / 4), c = (i % (kRtK / 4)) * 4;
-            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t0 + r < T) xv = load_act4<kBf16>(static_cast<const char*>(x) + (size_t)(t0 + r) * H * (kBf16 ? 2 : 4), k0 + c);
-            if (e0 + r < E) wv = *reinterpret_cast<const float4*>(w_router + (size_t)(e0 + r) * H + k0 + c);
-            xs[c][r] = xv.x; xs[c + 1][r] = xv.y; xs[c + 2][r] = xv.z; xs[c + 3][r] = xv.w;
-            ws[c][r] = wv.x; ws[c + 1][r] = wv.y; ws[c + 2][r] = wv.z; ws[c + 3][r] = wv.w;
+    __shared__ __align__(16) float xs[2][kRtK][kRtT + 4];
+    __shared__ __align__(16) float ws[2][kRtK][kRtE + 4];
+    const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;  // outputs (t0 + ty*8 + i, e0 + tx*4 + j)
+    // global -> register staging: x rows (tid & 127), k chunks of 4; w rows (tid & 63)
+    const int xr = tid & 127, xk = (tid >> 7) * 4;   // x: k = xk + 8 q, q < 2
+    const int wr = tid & 63, wk = (tid >> 6) * 4;    // w: k = wk
+    const size_t xrow_bytes = (size_t)H * (kBf16 ? 2 : 4);
+    const bool xin = t0 + xr < T, win = e0 + wr < E;
+    const char* xp = static_cast<const char*>(x) + (size_t)(xin ? t0 + xr : 0) * xrow_bytes;
+    const float* wp = w_router + (size_t)(win ? e0 + wr : 0) * H;
+    float4 xv[2], wv;
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            xv[q] = xin ? load_act4<kBf16>(xp, k0 + xk + 8 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        wv = win ? *reinterpret_cast<const float4*>(wp + k0 + wk) : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int k = xk + 8 * q;
+            xs[buf][k][xr] = xv[q].x;
+            xs[buf][k + 1][xr] = xv[q].y;
+            xs[buf][k + 2][xr] = xv[q].z;
+            xs[buf][k + 3][xr] = xv[q].w;
         }
-        __syncthreads();
-#pragma unroll 8
+        ws[buf][wk][wr] = wv.x;
+        ws[buf][wk + 1][wr] = wv.y;
+        ws[buf][wk + 2][wr] = wv.z;
+        ws[buf][wk + 3][wr] = wv.w;
+    };
+    float2 acc[8][2];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+    fetch(0);
+    store(0);
+    __syncthreads();
+    const int nk = H / kRtK;
+    for (int ks = 0; ks < nk; ++ks) {
+        const int buf = ks & 1;
+        if (ks + 1 < nk) fetch((ks + 1) * kRtK);
+#pragma unroll
         for (int kk = 0; kk < kRtK; ++kk) {
-            const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-            const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+            const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 8]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 8 + 4]);
+            const float4 bw = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float2 b01 = make_float2(bw.x, bw.y), b23 = make_float2(bw.z, bw.w);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            for (int i = 0; i < 8; ++i) {
+                const float2 ai = make_float2(av[i], av[i]);
+                acc[i][0] = __ffma2_rn(ai, b01, acc[i][0]);
+                acc[i][1] = __ffma2_rn(ai, b23, acc[i][1]);
+            }
         }
+        if (ks + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + ty * 8 + i;
+        if (t >= T) continue;
+        const float o[4] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
-            if (t < T && e < E) logits[(size_t)t * E + e] = acc[i][j];
+            const int e = e0 + tx * 4 + j;
+            if (e < E) logits[(size_t)t * E + e] = o[j];
         }
+    }
+}
+
+// Routing weights of a warp's top-k: lane j < k holds slot j's expert my_e and
+// its unbiased sigmoid my_s.  w_j = routed_scale * s_j / sum s.  With adaptive
+// expert top-p (0 < top_p < 1; "colibri解説", section 速度を稼ぐ実用ノブ, --topp):
+// the slots are ranked by share s_j / sum s (descending, lower expert first), a
+// slot is kept while the share of the slots ranked ahead of it is below top_p
+// (the shortest prefix that reaches top_p), the kept weights are renormalised
+// over the kept slots and a dropped slot gets expert -1 and weight 0.  Every
+// sum runs in slot order; without top-p the result is the plain weights.
+__device__ __forceinline__ void topk_weights(int k, float top_p, float routed_scale, int& my_e, float my_s,
+                                             float& my_w)
+{
+    const int lane = threadIdx.x & 31;
+    float total = 0.f;
+    for (int j = 0; j < k; ++j) total += __shfl_sync(0xFFFFFFFFu, my_s, j);
+    bool keep = lane < k;
+    if (top_p > 0.f && top_p < 1.f) {
+        float ahead = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const float sj = __shfl_sync(0xFFFFFFFFu, my_s, j);
+            const int ej = __shfl_sync(0xFFFFFFFFu, my_e, j);
+            if (j != lane && (sj > my_s || (sj == my_s && ej < my_e))) ahead += sj;
+        }
+        keep = keep && ahead / total < top_p;
+    }
+    float kept = 0.f;
+    for (int j = 0; j < k; ++j) kept += __shfl_sync(0xFFFFFFFFu, keep ? my_s : 0.f, j);
+    my_w = keep ? routed_scale * my_s / kept : 0.f;
+    if (lane < k && !keep) my_e = -1;
 }
 
 // Top-k of one token by one warp: sigmoid, bias, k rounds of warp arg-max,
@@ -133,7 +203,7 @@ router_logits_tiled_kernel(const void* __restrict__ x, int T, int H, const float
 // kPer = experts held per lane (E <= 32 * kPer).
 template <int kPer>
 __device__ __forceinline__ void topk_warp_rounds(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
-                                            float routed_scale, int32_t* idx_row, float* w_row)
+                                            float routed_scale, float top_p, int32_t* idx_row, float* w_row)
 {
     const int lane = threadIdx.x & 31;
     float s[kPer], c[kPer];
@@ -183,11 +253,11 @@ __device__ __forceinline__ void topk_warp_rounds(const float* lrow, int E, int k
             my_s = bs;
         }
     }
-    float total = 0.f;
-    for (int j = 0; j < k; ++j) total += __shfl_sync(0xFFFFFFFFu, my_s, j);
+    float my_w;
+    topk_weights(k, top_p, routed_scale, my_idx, my_s, my_w);
     if (lane < k) {
         idx_row[lane] = my_idx;
-        w_row[lane] = routed_scale * my_s / total;
+        w_row[lane] = my_w;
     }
 }
 
@@ -200,7 +270,7 @@ __device__ __forceinline__ void topk_warp_rounds(const float* lrow, int E, int k
 // that owns it pops its head.
 template <int kPer>
 __device__ __forceinline__ void topk_warp_heads(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
-                                                float routed_scale, int32_t* idx_row, float* w_row)
+                                                float routed_scale, float top_p, int32_t* idx_row, float* w_row)
 {
     const int lane = threadIdx.x & 31;
     unsigned long long key[kPer];
@@ -241,13 +311,13 @@ __device__ __forceinline__ void topk_warp_heads(const float* lrow, int E, int k,
         }
         if (lane == j) mine = best;
     }
-    const int my_e = (int)(0xFFFFu - (uint32_t)(mine & 0xFFFFu));
+    int my_e = (int)(0xFFFFu - (uint32_t)(mine & 0xFFFFu));
     const float my_s = lane < k ? 1.0f / (1.0f + expf(-lrow[my_e])) : 0.f;
-    float total = 0.f;
-    for (int j = 0; j < k; ++j) total += __shfl_sync(0xFFFFFFFFu, my_s, j);
+    float my_w;
+    topk_weights(k, top_p, routed_scale, my_e, my_s, my_w);
     if (lane < k) {
         idx_row[lane] = my_e;
-        w_row[lane] = routed_scale * my_s / total;
+        w_row[lane] = my_w;
     }
 }
 
@@ -255,17 +325,17 @@ __device__ __forceinline__ void topk_warp_heads(const float* lrow, int E, int k,
 // lane, rounds of arg-max above that.
 template <int kPer>
 __device__ __forceinline__ void topk_warp_t(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
-                                            float routed_scale, int32_t* idx_row, float* w_row)
+                                            float routed_scale, float top_p, int32_t* idx_row, float* w_row)
 {
-    if constexpr (kPer <= 8) topk_warp_heads<kPer>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
-    else topk_warp_rounds<kPer>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
+    if constexpr (kPer <= 8) topk_warp_heads<kPer>(lrow, E, k, sel_bias, routed_scale, top_p, idx_row, w_row);
+    else topk_warp_rounds<kPer>(lrow, E, k, sel_bias, routed_scale, top_p, idx_row, w_row);
 }
 
 __device__ __forceinline__ void topk_warp(const float* lrow, int E, int k, const float* __restrict__ sel_bias,
-                                          float routed_scale, int32_t* idx_row, float* w_row)
+                                          float routed_scale, float top_p, int32_t* idx_row, float* w_row)
 {
-    if (E <= 256) topk_warp_t<8>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
-    else topk_warp_t<kMaxExperts / 32>(lrow, E, k, sel_bias, routed_scale, idx_row, w_row);
+    if (E <= 256) topk_warp_t<8>(lrow, E, k, sel_bias, routed_scale, top_p, idx_row, w_row);
+    else topk_warp_t<kMaxExperts / 32>(lrow, E, k, sel_bias, routed_scale, top_p, idx_row, w_row);
 }
 
 // One warp per token, logits from global memory (layer path).  When launched as
@@ -273,14 +343,14 @@ __device__ __forceinline__ void topk_warp(const float* lrow, int E, int k, const
 // dependent launch at once (that kernel waits for this one's results).
 __global__ void __launch_bounds__(256)
 router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                   const float* __restrict__ sel_bias, float routed_scale,
+                   const float* __restrict__ sel_bias, float routed_scale, float top_p,
                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w)
 {
     griddep_wait();
     griddep_launch_dependents();
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;  // whole warp leaves together
-    topk_warp(logits + (size_t)t * E, E, k, sel_bias, routed_scale, topk_idx + (size_t)t * k,
+    topk_warp(logits + (size_t)t * E, E, k, sel_bias, routed_scale, top_p, topk_idx + (size_t)t * k,
               topk_w + (size_t)t * k);
 }
 
@@ -336,7 +406,7 @@ router_cluster_kernel(const void* __restrict__ x, int T, int H, const float* __r
     }
     cluster.sync();
     if (rank == 0 && warp < nt)
-        topk_warp(&s_logits[warp][0], E, k, sel_bias, routed_scale, topk_idx + (size_t)(t0 + warp) * k,
+        topk_warp(&s_logits[warp][0], E, k, sel_bias, routed_scale, 0.f, topk_idx + (size_t)(t0 + warp) * k,
                   topk_w + (size_t)(t0 + warp) * k);
 }
 

@@ -92,3 +92,18 @@ def output_to_f64(out, torch):
     if out.dtype == torch.bfloat16:
         return out.float().cpu().numpy().astype(np.float64)
     return out.cpu().numpy().astype(np.float64)
+
+
+def near_top_p_boundary(x, w_router, sel_bias, k, alpha, top_p, gap=GAP):
+    """Tokens where some prefix of the selected experts' routing shares (largest
+    first) sums to within `gap` of top_p: the cut there is decided by rounding,
+    and the oracle (f64) and the kernels (fp32) may cut differently."""
+    idx, _, (_, sig, _) = oracle.route(x, w_router, sel_bias, k, alpha, want_scores=True)
+    bad = []
+    for t in range(idx.shape[0]):
+        s = sig[t, idx[t]]
+        order = np.lexsort((idx[t], -s))  # share descending, lower expert first
+        cum = np.cumsum(s[order] / s.sum())
+        if np.any(np.abs(cum - top_p) < gap):
+            bad.append(t)
+    return np.array(bad, np.int64)

@@ -75,26 +75,24 @@ def test_workspace_size_is_positive_and_grows(coli):
 
 def test_status_word_offset(coli):
     """The device status word sits inside the workspace of the call it belongs
-    to, 4-byte aligned; calls that do not write it (one-token chain, empty
-    batches, invalid layers) report none."""
+    to, 4-byte aligned; calls that do not write it (empty batches, invalid
+    layers) report none."""
     none = ctypes.c_size_t(-1).value
     lib = coli.lib()
     s = _layer(coli)
-    for T in (2, 4, 64, 65, 4096):
+    for T in (1, 2, 4, 64, 65, 4096):
         off = lib.coli_moe_status_word_offset(ctypes.byref(s), T)
         assert off != none and off % 4 == 0
         assert off + 4 <= lib.coli_moe_workspace_size(ctypes.byref(s), T)
-    assert lib.coli_moe_status_word_offset(ctypes.byref(s), 1) == none  # one-token chain
     assert lib.coli_moe_status_word_offset(ctypes.byref(s), 0) == none
     assert lib.coli_moe_status_word_offset(None, 4) == none
     assert lib.coli_moe_status_word_offset(ctypes.byref(_layer(coli, hidden=100)), 4) == none
-    # one token of another shape goes through the union, which writes the word
     small = _layer(coli, hidden=1024, ffn=512, n_experts=64)
     assert lib.coli_moe_status_word_offset(ctypes.byref(small), 1) != none
     # the Python binding maps "none" to None
     L = coli.Layer.__new__(coli.Layer)
     L.struct = s
-    assert coli.moe_status_word_offset(L, 1) is None
+    assert coli.moe_status_word_offset(L, 0) is None
     assert coli.moe_status_word_offset(L, 4) == lib.coli_moe_status_word_offset(ctypes.byref(s), 4)
 
 
@@ -102,7 +100,7 @@ def test_status_word_offset(coli):
     (dict(hidden=100), 1), (dict(hidden=0), 1), (dict(ffn=96), 1), (dict(top_k=0), 1),
     (dict(top_k=33), 1), (dict(n_experts=4, top_k=8), 1), (dict(n_experts=2000), 1),
     (dict(group=128), 2), (dict(hidden=32768), 2), (dict(w_router=0), 1), (dict(gate_q=(1 << 20) + 8), 1),
-    (dict(routed_scale=float("inf")), 1),
+    (dict(routed_scale=float("inf")), 1), (dict(top_p=-0.5), 1), (dict(top_p=float("nan")), 1),
 ])
 def test_forward_rejects_bad_layers(coli, over, status):
     assert _fwd(coli, _layer(coli, **over)) == status
@@ -157,12 +155,21 @@ def test_path_choice(coli):
     assert [coli.moe_path(L, T) for T in (0, 1, 2, 64, 65, 4096)] == \
         ["none", "single", "decode", "decode", "prefill", "prefill"]
     L.struct = _layer(coli, hidden=256, ffn=128, n_experts=16, top_k=4)
-    assert coli.moe_path(L, 130) == "decode"  # ffn not a multiple of 256: CUDA cores at any batch
-    assert coli.moe_path(L, 1) == "decode"    # one token of another shape
+    assert coli.moe_path(L, 130) == "wide"    # ffn not a multiple of 256: CUDA-core expert phases
+    assert coli.moe_path(L, 1) == "single"
+    assert coli.moe_path(L, 64) == "decode"
+    # the decode kernel's shared memory (activations, union tables) does not fit: expert phases
+    L.struct = _layer(coli, hidden=16384, ffn=16384, n_experts=1024, top_k=32)
+    assert coli.moe_path(L, 64) == "wide"
     L.struct = _layer(coli, hidden=256, ffn=256, n_experts=16, top_k=4)
     assert coli.moe_path(L, 130) == "prefill"
     L.struct = _layer(coli, hidden=100)
     assert coli.moe_path(L, 4) == "none"
+
+
+def test_wait_limit_hook_takes_any_value(coli):
+    coli.debug_set_wait_ns(1000)
+    coli.debug_set_wait_ns(0)  # the built-in limit again
 
 
 def test_profile_hook_arms_and_disarms(coli):

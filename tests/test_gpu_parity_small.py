@@ -145,7 +145,7 @@ def test_ragged_batches(env, T):
     # ffn 128 is not a multiple of 256: every batch, 130 tokens included, runs on CUDA cores in fp32
     coli, torch = env
     L = S.upload_layer(coli, torch, c, w_router, sel_bias, inputs.stack_experts(ex, c.E))
-    assert coli.moe_path(L, T) == "decode"
+    assert coli.moe_path(L, T) == ("single" if T == 1 else "decode" if T <= 64 else "wide")
     S.check_output(out, rout, S.TOL_DECODE, f"ragged T={T}")
 
 
