@@ -162,13 +162,33 @@ constexpr int kSlotBytes = 32 * (16 + 16 + 4 + 4);  // one step of a warp: two 1
 // hook(): called by every thread once the first R - 1 steps are in flight and
 // before the first one is consumed (e.g. a barrier and the staging of the
 // vectors), also by warps that have no items.
-__device__ __forceinline__ void cp_async16_s(uint32_t smem, const void* gmem)
+// The streamed weights are read once per call: they are copied with an
+// evict-first L2 policy, so that the stream (far larger than L2) does not push
+// the kernel's instructions and the call's small shared data (activations,
+// router partials, h) out of L2 between and within calls.
+__device__ __forceinline__ uint64_t l2_evict_first()
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem), "l"(gmem) : "memory");
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
 }
-__device__ __forceinline__ void cp_async4_s(uint32_t smem, const void* gmem)
+__device__ __forceinline__ void cp_async16_s(uint32_t smem, const void* gmem, uint64_t pol)
 {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem), "l"(gmem) : "memory");
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem), "l"(gmem), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4_s(uint32_t smem, const void* gmem, uint64_t pol)
+{
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 4, %2;" ::"r"(smem), "l"(gmem), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ float4 ldg_stream4(const float4* p, uint64_t pol)
+{
+    float4 v;
+    asm("ld.global.nc.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
 }
 __device__ __forceinline__ uint4 lds128(uint32_t smem)
 {
@@ -198,6 +218,7 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
     const uint32_t ring_lane = smem_u32(ring) + lane * 16;
     const uint32_t ring_end = ring_lane + R * kSlotBytes;
     const uint32_t sc_off = 1024 - 12 * lane;
+    const uint64_t pol = l2_evict_first();
     // load cursor: item lj (0-based among mine), chunk step lci, this lane's slot address and source pointers
     int lj = 0, lci = 0;
     uint32_t lsl = ring_lane;
@@ -214,10 +235,10 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
     set_rows(j0);
     auto issue = [&]() {
         if (lj < nj && (whole || lane + 32 * lci < nch)) {
-            cp_async16_s(lsl, pq0);
-            cp_async16_s(lsl + 512, pq1);
-            cp_async4_s(lsl + sc_off, ps0);
-            cp_async4_s(lsl + sc_off + 128, ps1);
+            cp_async16_s(lsl, pq0, pol);
+            cp_async16_s(lsl + 512, pq1, pol);
+            cp_async4_s(lsl + sc_off, ps0, pol);
+            cp_async4_s(lsl + sc_off + 128, ps1, pol);
         }
         cp_async_commit();  // one group per step (empty past the end)
         pq0 += 512;         // this lane's next chunk: 32 chunks on
@@ -310,10 +331,10 @@ struct LayerArgs {
 
 constexpr int kStamps = 16;
 
-// Test hook: thread 0 of each CTA records the time it reached point i.
-__device__ __forceinline__ void stamp(const LayerArgs& a, int i)
+// Test hook: thread `by` (default 0) of each CTA records the time it reached point i.
+__device__ __forceinline__ void stamp(const LayerArgs& a, int i, int by = 0)
 {
-    if (a.stamps && threadIdx.x == 0) a.stamps[blockIdx.x * kStamps + i] = layer_ns();
+    if (a.stamps && threadIdx.x == by) a.stamps[blockIdx.x * kStamps + i] = layer_ns();
 }
 
 // Shared-memory plan of one launch (host and device compute the same one).
@@ -442,74 +463,96 @@ namespace coli {
 
 // Top-k of one token by one warp; lane l holds the router scores of experts
 // e = l + 32 i in l[i] (E <= 32 kPer).  Same rule as the layer's other top-k:
-// key = order-preserving image of c = sigmoid(logit) + bias (NaN -> -inf,
-// -0 -> +0) then the complement of the index, so larger keys mean (c desc,
-// index asc) and keys are unique.  Each lane sorts its keys (carrying the
-// unbiased sigmoid along); k rounds take the warp maximum of the heads, the
-// owner pops its head and hands out its sigmoid.  Lane j < k returns expert
-// and weight routed_scale * s_j / sum s.
+// order by c = sigmoid(logit) + bias descending (NaN -> -inf, -0 -> +0), ties
+// to the lower expert index.  c is mapped to an order-preserving 32-bit key
+// (never 0 for an expert; 0 marks an empty or taken entry).  Each round every
+// lane offers its best remaining entry (lowest index among equal keys), a warp
+// max-reduction picks the key and a min-reduction over the lanes offering it
+// picks the lowest expert index; the owner marks it taken.  Lane j < k returns
+// the j-th expert and its weight routed_scale * s_j / sum s.
 template <int kPer>
 __device__ __forceinline__ void topk_regs(const float (&l)[kPer], int E, int k, const float* __restrict__ sel_bias,
                                           float routed_scale, float top_p, int& my_e, float& my_w)
 {
     const int lane = threadIdx.x & 31;
-    unsigned long long key[kPer];
+    uint32_t key[kPer];
     float sg[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
-        key[i] = 0ull;
+        key[i] = 0u;
         sg[i] = 0.f;
         if (e < E) {
             const float s = 1.0f / (1.0f + expf(-l[i]));
             const float ci = s + sel_bias[e];
             const float c = (ci == ci) ? ci + 0.0f : -INFINITY;
             const uint32_t u = __float_as_uint(c);
-            const uint32_t m = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-            key[i] = ((unsigned long long)m << 32) | (uint32_t)(0xFFFFu - e);
+            key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
             sg[i] = s;
         }
     }
-#pragma unroll
-    for (int r = 0; r < kPer; ++r)
-#pragma unroll
-        for (int i = r & 1; i + 1 < kPer; i += 2) {
-            const bool sw = key[i] < key[i + 1];
-            const unsigned long long a = key[i], b = key[i + 1];
-            const float sa = sg[i], sb = sg[i + 1];
-            key[i] = sw ? b : a;
-            key[i + 1] = sw ? a : b;
-            sg[i] = sw ? sb : sa;
-            sg[i + 1] = sw ? sa : sb;
-        }
     my_e = -1;
     float my_s = 0.f;
     for (int j = 0; j < k; ++j) {
-        unsigned long long best = key[0];
+        uint32_t bk = 0u;
+        int bi = 0;
+        float bs = 0.f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-            best = other > best ? other : best;
-        }
-        const int e = (int)(0xFFFFu - (uint32_t)(best & 0xFFFFu));
-        float popped = 0.f;
-        if (key[0] == best) {  // the unique owner (lane e % 32) pops its head
-            popped = sg[0];
-#pragma unroll
-            for (int i = 0; i + 1 < kPer; ++i) {
-                key[i] = key[i + 1];
-                sg[i] = sg[i + 1];
+        for (int i = 0; i < kPer; ++i)
+            if (key[i] > bk) {
+                bk = key[i];
+                bi = i;
+                bs = sg[i];
             }
-            key[kPer - 1] = 0ull;
-            sg[kPer - 1] = 0.f;
+        const uint32_t top = __reduce_max_sync(0xFFFFFFFFu, bk);
+        const uint32_t e = __reduce_min_sync(0xFFFFFFFFu, bk == top ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu);
+        const float s = __shfl_sync(0xFFFFFFFFu, bs, e & 31);
+        if (lane == (int)(e & 31)) {
+#pragma unroll
+            for (int i = 0; i < kPer; ++i)
+                if (i == (int)(e >> 5)) key[i] = 0u;
         }
-        const float s = __shfl_sync(0xFFFFFFFFu, popped, e & 31);
         if (lane == j) {
-            my_e = e;
+            my_e = (int)e;
             my_s = s;
         }
     }
     topk_weights(k, top_p, routed_scale, my_e, my_s, my_w);
+}
+
+// Top-k of one token by one warp from per-expert selection keys in shared
+// memory (key as in topk_regs, 0 = taken).  Each round every lane offers its
+// best remaining expert (lowest index among equal keys), a max-reduction picks
+// the key, a min-reduction the lowest index offering it, and lane 0 clears it.
+// Lane j < k returns the j-th expert and its sigmoid; the loops are rolled (the
+// code runs once per call).
+__device__ __forceinline__ void topk_smem(uint32_t* key, const float* sig, int E, int k, int& my_e, float& my_s)
+{
+    const int lane = threadIdx.x & 31;
+    my_e = -1;
+    my_s = 0.f;
+    for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0u;
+        int be = 0;
+#pragma unroll 4
+        for (int e = lane; e < E; e += 32) {
+            const uint32_t kv = key[e];
+            if (kv > bk) {
+                bk = kv;
+                be = e;
+            }
+        }
+        const uint32_t top = __reduce_max_sync(0xFFFFFFFFu, bk);
+        const uint32_t e = __reduce_min_sync(0xFFFFFFFFu, bk == top ? (uint32_t)be : 0xFFFFFFFFu);
+        if (e < (uint32_t)E) {
+            if (lane == 0) key[e] = 0u;
+            if (lane == j) {
+                my_e = (int)e;
+                my_s = sig[e];
+            }
+        }
+        __syncwarp();
+    }
 }
 
 // Top-k of token t for more than 256 experts (same rule and result as
@@ -722,9 +765,10 @@ __device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, i
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
     if (c < g.nch) {
         const float4* wrow = reinterpret_cast<const float4*>(a.w_router + (size_t)e * a.H) + (size_t)c * 8;
+        const uint64_t pol = l2_evict_first();
         float4 wv[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) wv[j] = __ldg(wrow + j);
+        for (int j = 0; j < 8; ++j) wv[j] = ldg_stream4(wrow + j, pol);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             if (t < nt) {
@@ -788,11 +832,12 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const bool all_x = T <= MT;  // every token's activations staged once for the whole call
     const int n_sg = (T + MT - 1) / MT;  // shared-expert groups
 
-    auto stage_x = [&](int n, auto token_of) {
-        stage_vectors<kBf16>(a.x, H, n, token_of, gH, xs, xcorr);
+    // activations / SwiGLU outputs into shared memory: vector t = row row0 + t (or tbl[t] / tdiv)
+    auto stage_x = [&](int n, int row0, const int* tbl = nullptr, int tdiv = 1) {
+        stage_rows(a.x, kBf16 ? 1 : 0, H, n, row0, tbl, tdiv, xs, xcorr, (int)threadIdx.x, kLayerThreads);
     };
-    auto stage_h = [&](int n, auto pos_of) {
-        stage_vectors<false>(a.h, F, n, pos_of, gF, hs, hcorr);
+    auto stage_h = [&](int n, int row0) {
+        stage_rows(a.h, 0, F, n, row0, nullptr, 1, hs, hcorr, (int)threadIdx.x, kLayerThreads);
     };
 
     // gate/up item finisher: h[pos_t, n] = silu(gate) * up for the group's vectors
@@ -822,7 +867,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 router_piece<MT>(a, i / nrp, i % nrp, T, gH, xs);
         };
         auto stage_all = [&]() {
-            stage_x(T, [](int t) { return t; });
+            stage_x(T, 0);
             __syncthreads();
             stamp(a, 1);
         };
@@ -835,6 +880,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const SegTable st = seg_prepare(u, nseg);
         int lo, hi;
         seg_cta_range(st, lo, hi);
+        stamp(a, 10);
         bool ran = false;
         for (int s = 0; s < nseg; ++s) {
             const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
@@ -868,7 +914,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     }
                 } else {  // this group's tokens (the router ran before the launch)
                     __syncthreads();
-                    stage_x(m, [t0](int t) { return t0 + t; });
+                    stage_x(m, t0);
                     __syncthreads();
                 }
             };
@@ -905,50 +951,64 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         __syncthreads();
     };
     if constexpr (kOutRows) {
-        sum_pieces();
-        if (warp == 0) {
-            // the token's top-k, then the union of its k experts: ascending expert order
-            int my_e;
-            float my_w;
-            if (E <= 256) {
-                float l[8];
+        // The shared expert's down rows for this CTA's output rows need no routing: their first
+        // loads are issued, then (hook) the token is scored and routed by warp 0 while the other
+        // warps stage h of the shared expert; no warp streams while the route is taken.
+        auto route_hook = [&]() {
+            // the token's router scores (sums of the pieces), sigmoids and selection keys
+            uint32_t* s_key = reinterpret_cast<uint32_t*>(u.mask);  // the union's token masks are not used here
+            float* s_sig = reinterpret_cast<float*>(u.mask) + E;
+            for (int e = threadIdx.x; e < E; e += kLayerThreads) {
+                float v = 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int e = lane + 32 * i;
-                    l[i] = e < E ? s_logit[e] : 0.f;
+                for (int p = 0; p < 16; ++p)
+                    if (p < npc) v += a.logit_part[(size_t)p * E + e];
+                const float sg = 1.0f / (1.0f + expf(-v));
+                const float ci = sg + a.sel_bias[e];
+                const float c = (ci == ci) ? ci + 0.0f : -INFINITY;
+                const uint32_t cu = __float_as_uint(c);
+                s_key[e] = (cu & 0x80000000u) ? ~cu : (cu | 0x80000000u);
+                s_sig[e] = sg;
+            }
+            __syncthreads();
+            stamp(a, 11);
+            if (warp == 0) {
+                // the token's top-k, then the union of its k experts: ascending expert order
+                int my_e;
+                float my_s, my_w;
+                topk_smem(s_key, s_sig, E, k, my_e, my_s);
+                topk_weights(k, a.top_p, a.routed_scale, my_e, my_s, my_w);
+                // kept experts (top-p may drop slots: expert -1) in ascending order
+                int rank = 0;
+                for (int i = 0; i < k; ++i) {
+                    const int ei = __shfl_sync(0xFFFFFFFFu, my_e, i);
+                    rank += (ei >= 0 && ei < my_e) ? 1 : 0;
                 }
-                topk_regs<8>(l, E, k, a.sel_bias, a.routed_scale, a.top_p, my_e, my_w);
+                const int n_kept = __popc(__ballot_sync(0xFFFFFFFFu, lane < k && my_e >= 0));
+                if (lane < k) {
+                    u.idx[lane] = my_e;
+                    u.w[lane] = my_w;
+                    u.ipos[lane] = my_e >= 0 ? rank : -1;
+                    if (my_e >= 0) {
+                        u.perm[rank] = lane;
+                        u.gexp[rank] = my_e;
+                        u.gpos[rank] = rank;
+                    }
+                    if (blockIdx.x == 0) {
+                        a.idx_out[lane] = my_e;
+                        a.w_out[lane] = my_w;
+                    }
+                }
+                if (lane == 0) reinterpret_cast<int*>(u.tmp)[0] = n_kept;
+                stamp(a, 12);
             } else {
-                topk_rounds_global(a.logit_part, npc, 1, 0, E, k, a.sel_bias, a.routed_scale, a.top_p, my_e, my_w);
+                stage_rows(a.h, 0, F, 1, P, nullptr, 1, hs + (size_t)k * gF.f4, hcorr + (size_t)k * gF.nch,
+                           (int)threadIdx.x - 32, kLayerThreads - 32);
+                stamp(a, 13, 32);
             }
-            // kept experts (top-p may drop slots: expert -1) in ascending order
-            int rank = 0;
-            for (int i = 0; i < k; ++i) {
-                const int ei = __shfl_sync(0xFFFFFFFFu, my_e, i);
-                rank += (ei >= 0 && ei < my_e) ? 1 : 0;
-            }
-            const int n_kept = __popc(__ballot_sync(0xFFFFFFFFu, lane < k && my_e >= 0));
-            if (lane < k) {
-                u.idx[lane] = my_e;
-                u.w[lane] = my_w;
-                u.ipos[lane] = my_e >= 0 ? rank : -1;
-                if (my_e >= 0) {
-                    u.perm[rank] = lane;
-                    u.gexp[rank] = my_e;
-                    u.gpos[rank] = rank;
-                }
-                if (blockIdx.x == 0) {
-                    a.idx_out[lane] = my_e;
-                    a.w_out[lane] = my_w;
-                }
-            }
-            if (lane == 0) reinterpret_cast<int*>(u.tmp)[0] = n_kept;
-        } else {
-            // meanwhile: the shared expert's h, and its down rows for this CTA's output rows
-            const int tid = threadIdx.x - 32, nthr = kLayerThreads - 32;
-            stage_vectors<false>(a.h, F, 1, [&](int) { return P; }, gF, hs + (size_t)k * gF.f4, hcorr + (size_t)k * gF.nch,
-                                 tid, nthr);
-            asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+            __syncthreads();
+        };
+        {
             auto rows_of = [&](int j, RowPair& r) {
                 const size_t row = (size_t)E * H + 2 * (pr_lo + j);
                 r.q0 = a.down_q + row * (F / 2);
@@ -971,11 +1031,12 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     ypart[(2 * j + 1) * S1 + k] = y1;
                 }
             };
-            const int first = warp - 1, nw = kLayerWarps - 1;
-            const int nj = first < npr ? (npr - first + nw - 1) / nw : 0;
-            stream_row_pairs<MT, P_DN>(first, nw, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin);
+            const int first = warp;
+            const int nj = first < npr ? (npr - first + kLayerWarps - 1) / kLayerWarps : 0;
+            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of,
+                                       fin, route_hook);
         }
-        __syncthreads();
+        stamp(a, 14);
         stamp(a, 4);
         // routed gate/up: the kept experts x F rows, equal cost, an even split
         const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
@@ -1099,7 +1160,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             if (s_lo >= s_hi) continue;
             const int t0 = s * MT, m = min(MT, T - t0);
             __syncthreads();
-            stage_h(m, [&](int t) { return P + t0 + t; });
+            stage_h(m, P + t0);
             __syncthreads();
             const int base = st.ipre[s];
             auto rows_of = [&](int j, RowPair& r) {
@@ -1152,7 +1213,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 const int g = s - n_sd, e = u.gexp[g], p0 = u.gpos[g];
                 const int m = min(MT, u.off[e] + u.cnt[e] - p0);
                 __syncthreads();
-                stage_x(m, [&](int t) { return u.perm[p0 + t] / k; });
+                stage_x(m, 0, u.perm + p0, k);
                 __syncthreads();
             }
             auto seg_of = [&](int j) { return all_x ? last_le(st.ipre, nseg - 1, j) : s; };
@@ -1226,7 +1287,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         auto hook = [&]() {
             grid_barrier(bar, deadline, a.err);
             stamp(a, 6);
-            stage_h(n_kept, [&](int g) { return g; });  // h of the g-th kept expert sits at position g
+            stage_h(n_kept, 0);  // h of the g-th kept expert sits at position g
             __syncthreads();
             stamp(a, 7);
         };
@@ -1266,7 +1327,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             const int e = u.gexp[s], p0 = u.gpos[s];
             const int m = min(MT, u.off[e] + u.cnt[e] - p0);
             __syncthreads();
-            stage_h(m, [&](int t) { return p0 + t; });
+            stage_h(m, p0);
             __syncthreads();
             const int base = st.ipre[s];
             auto rows_of = [&](int j, RowPair& r) {
