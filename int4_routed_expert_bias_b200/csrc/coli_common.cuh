@@ -19,6 +19,35 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
+// Sums of a and b over the warp in five exchanges: lane 0 ends with the sum of
+// a, lane 16 with the sum of b.
+__device__ __forceinline__ float warp_sum2(float a, float b)
+{
+    const bool hi = (threadIdx.x & 16) != 0;
+    float v = (hi ? b : a) + __shfl_xor_sync(0xFFFFFFFFu, hi ? a : b, 16);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// floor(j / d) for 0 <= j <= j_max by a divisor fixed for the call: the high
+// word of j * ceil(2^32 / d), exact while j_max * d < 2^32 (else a plain
+// division is used).
+struct FastDiv {
+    uint32_t m;  // ceil(2^32 / d) (0 when d == 1)
+    int d;
+    bool exact;
+    __device__ __forceinline__ FastDiv(int d_, long long j_max)
+        : m(d_ > 1 ? (uint32_t)((0x100000000ull + (unsigned long long)d_ - 1ull) / (unsigned long long)d_) : 0u),
+          d(d_), exact((unsigned long long)j_max * (unsigned long long)d_ < 0x100000000ull)
+    {
+    }
+    __device__ __forceinline__ int operator()(int j) const
+    {
+        return !exact ? j / d : m ? (int)__umulhi((uint32_t)j, m) : j;
+    }
+};
+
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
 // fp32 -> bf16 bits, round to nearest even (inputs here are finite).

@@ -227,6 +227,191 @@ static __device__ __noinline__ void stage_rows(const void* __restrict__ src, int
     }
 }
 
+// ---------------------------------------------------------------------------
+// Integer-dot form of the one-vector products.
+//
+// An activation chunk of 32 values is held as 21-bit fixed point over one
+// power-of-two chunk scale: with m = max |x| < 2^e,
+//   X = round(x * 2^(21 - e)),  |X| < 2^21,   x_hat = 2^(e - 21) X,
+// so |x - x_hat| <= 2^(e - 22) <= 2^-21 m.  X is stored as three 8-bit digit
+// planes, its two's-complement bit slices X = 16384 d0 + 128 d1 + d2 (d0 the
+// signed top byte, d1 and d2 seven unsigned bits each).  An int4 word becomes
+// biased bytes n = q + 8 in [0, 15] with three integer operations (lo:
+// nibbles 0, 2, 4, 6; hi: nibbles 1, 3, 5, 7), and dp4a sums n * d exactly in
+// int32 per plane.  Per chunk and row:
+//   sum_k q_k x_hat_k = 2^(e - 21) * (D - corr),
+//   D = sum_k n_k X_k = 16384 D0 + 128 D1 + D2,  corr = 8 * sum_k X_k,
+// an exact integer below 2^29 in magnitude, converted to fp32 once.  The
+// integer products leave the float pipes free and take far fewer issue slots
+// than decoding nibbles to floats.
+//
+// Shared-memory layout of one staged vector: chunk c = l + 32 i, plane
+// p = 2 * digit + (0: lo, 1: hi), as uint4 at ((i * 6 + p) * 32 + l); word w
+// of the uint4 covers k = 8 w .. 8 w + 7 of the chunk, byte b of a lo (hi)
+// word holds the digit of k = 8 w + 2 b (+ 1).  Per chunk one float2:
+// (2^(e - 21), corr as int bits).
+constexpr int kDigitPlanes = 6;
+
+__host__ __device__ inline int digit_vec_units(int K)  // 16-byte units per staged vector
+{
+    return stage_geom(K).per_lane * kDigitPlanes * 32;
+}
+
+__host__ __device__ inline size_t digit_smem_bytes(int K, int n_vectors)
+{
+    return (size_t)n_vectors * digit_vec_units(K) * 16 + (size_t)n_vectors * (K / kChunkK) * 8;
+}
+
+// biased bytes q + 8 of nibbles 0, 2, 4, 6 (lo) and 1, 3, 5, 7 (hi) of a word
+__device__ __forceinline__ uint32_t nib_lo_u8(uint32_t w)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(w), "r"(0x0F0F0F0Fu), "r"(0x08080808u));
+    return d;
+}
+__device__ __forceinline__ uint32_t nib_hi_u8(uint32_t w) { return nib_lo_u8(w >> 4); }
+
+// c + sum of the four products of unsigned bytes of a and signed bytes of b
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// low bytes of a, b, c, d as one word (a in byte 0)
+__device__ __forceinline__ uint32_t pack_lo_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Stage n vectors of K values (rows of src, fp32 or bf16) as digit planes: vector
+// t is row row0 + t of src, or row tbl[t] / tdiv when tbl is given.  One thread
+// encodes one chunk.  Threads tid = 0 .. nthr-1 share the work.  Not inlined:
+// one copy of the code serves every call site.
+static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ src, int bf16, int K, int n, int row0,
+                                                      const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
+                                                      int nthr)
+{
+    const int nch = K / kChunkK;
+    const int vunits = digit_vec_units(K);
+    const size_t row_bytes = (size_t)K * (bf16 ? 2 : 4);
+    for (int idx = tid; idx < n * nch; idx += nthr) {
+        const int t = idx / nch, c = idx - t * nch;
+        const int row = tbl ? tbl[t] / tdiv : row0 + t;
+        const char* rp = static_cast<const char*>(src) + (size_t)row * row_bytes;
+        float x[32];
+        if (bf16) {
+            const uint4* p4 = reinterpret_cast<const uint4*>(rp + (size_t)c * kChunkK * 2);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v = p4[j];
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    x[8 * j + 2 * h] = bf16_bits_to_float(u[h] & 0xFFFFu);
+                    x[8 * j + 2 * h + 1] = bf16_bits_to_float(u[h] >> 16);
+                }
+            }
+        } else {
+            const float4* p4 = reinterpret_cast<const float4*>(rp + (size_t)c * kChunkK * 4);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 v = p4[j];
+                x[4 * j] = v.x;
+                x[4 * j + 1] = v.y;
+                x[4 * j + 2] = v.z;
+                x[4 * j + 3] = v.w;
+            }
+        }
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(x[j]));
+        const bool finite = m <= 3.402823466e38f;  // false for inf and NaN
+        const int ex = (int)(__float_as_uint(m) >> 23);
+        // chunks whose largest magnitude is below 2^-100 contribute nothing (their products are far below any
+        // fp32 rounding of the result); e = ex - 126 gives m < 2^e
+        const bool live = finite && ex >= 26;
+        const int e = live ? ex - 126 : 0;
+        const float mult = live ? __uint_as_float((uint32_t)(148 - e) << 23) : 0.f;  // 2^(21 - e)
+        uint32_t X[32];
+        int csum = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            // round(x * 2^(21 - e)) by the 1.5 * 2^23 addition (|product| < 2^21 + 1 keeps it exact)
+            const int v = __float_as_int(fmaf(x[j], mult, 12582912.0f)) - 0x4B400000;
+            const int vc = min(v, (1 << 21) - 1);  // a value rounding up to 2^21 is held at the top code
+            X[j] = (uint32_t)vc;
+            csum += vc;
+        }
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
+        uint32_t lo[4], hi[4];
+        // plane d2: bits 0-6; d1: bits 7-13; d0: bits 14-21 (signed)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            lo[w] = pack_lo_bytes(X[8 * w], X[8 * w + 2], X[8 * w + 4], X[8 * w + 6]) & 0x7F7F7F7Fu;
+            hi[w] = pack_lo_bytes(X[8 * w + 1], X[8 * w + 3], X[8 * w + 5], X[8 * w + 7]) & 0x7F7F7F7Fu;
+        }
+        base[4 * 32] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        base[5 * 32] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            lo[w] = pack_lo_bytes(X[8 * w] >> 7, X[8 * w + 2] >> 7, X[8 * w + 4] >> 7, X[8 * w + 6] >> 7) & 0x7F7F7F7Fu;
+            hi[w] = pack_lo_bytes(X[8 * w + 1] >> 7, X[8 * w + 3] >> 7, X[8 * w + 5] >> 7, X[8 * w + 7] >> 7) &
+                    0x7F7F7F7Fu;
+        }
+        base[2 * 32] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        base[3 * 32] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            lo[w] = pack_lo_bytes(X[8 * w] >> 14, X[8 * w + 2] >> 14, X[8 * w + 4] >> 14, X[8 * w + 6] >> 14);
+            hi[w] = pack_lo_bytes(X[8 * w + 1] >> 14, X[8 * w + 3] >> 14, X[8 * w + 5] >> 14, X[8 * w + 7] >> 14);
+        }
+        base[0 * 32] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        base[1 * 32] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        const float scale = !finite ? __int_as_float(0x7FC00000) : live ? __uint_as_float((uint32_t)(106 + e) << 23)
+                                                                          : 0.f;
+        xc[(size_t)t * nch + c] = make_float2(scale, __int_as_float(8 * csum));
+    }
+}
+
+// Row-pair products of one chunk against a digit-staged vector: acc[row] gets
+// 2^(e - 21)-scaled exact integer sums (see above).  xd: this lane's plane 0 of
+// the chunk (planes 32 uint4 apart); c: the chunk's (scale, corr).
+__device__ __forceinline__ void chunk_pair_digits(const uint4& w0, const uint4& w1, const uint4* xd, float2 c,
+                                                  float s0, float s1, float& tot0, float& tot1)
+{
+    uint32_t al[4], ah[4], bl[4], bh[4];  // each word decoded once, used by the three digit planes
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t a = q == 0 ? w0.x : q == 1 ? w0.y : q == 2 ? w0.z : w0.w;
+        const uint32_t b = q == 0 ? w1.x : q == 1 ? w1.y : q == 2 ? w1.z : w1.w;
+        al[q] = nib_lo_u8(a);
+        ah[q] = nib_hi_u8(a);
+        bl[q] = nib_lo_u8(b);
+        bh[q] = nib_hi_u8(b);
+    }
+    int a0[3] = {0, 0, 0}, a1[3] = {0, 0, 0};
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+        const uint4 xl = xd[(2 * d) * 32], xh = xd[(2 * d + 1) * 32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t l = q == 0 ? xl.x : q == 1 ? xl.y : q == 2 ? xl.z : xl.w;
+            const uint32_t h = q == 0 ? xh.x : q == 1 ? xh.y : q == 2 ? xh.z : xh.w;
+            a0[d] = dp4a_us(al[q], l, a0[d]);
+            a0[d] = dp4a_us(ah[q], h, a0[d]);
+            a1[d] = dp4a_us(bl[q], l, a1[d]);
+            a1[d] = dp4a_us(bh[q], h, a1[d]);
+        }
+    }
+    const uint32_t corr = (uint32_t)__float_as_int(c.y);
+    const uint32_t D0 = ((uint32_t)a0[0] * 128u + (uint32_t)a0[1]) * 128u + (uint32_t)a0[2] - corr;
+    const uint32_t D1 = ((uint32_t)a1[0] * 128u + (uint32_t)a1[1]) * 128u + (uint32_t)a1[2] - corr;
+    tot0 = fmaf(s0 * c.x, (float)(int)D0, tot0);
+    tot1 = fmaf(s1 * c.x, (float)(int)D1, tot1);
+}
+
 // The same with every thread of the block.
 template <typename Load4>
 __device__ __forceinline__ void stage_vectors_fn(int n, Load4 load, const StageGeom& g, float4* xs, float* corr)

@@ -64,25 +64,43 @@ __device__ __forceinline__ unsigned long long layer_ns()
 // word (zero-based, provided by the driver for cooperative launches).  CTA 0
 // adds 2^31 - (G - 1) and every other CTA 1, so bit 31 of the word flips
 // exactly when the last CTA arrives and the low bits return to where they
-// were.  Arrival releases and the poll acquires at GPU scope, so writes before
-// the barrier are visible after it.  Gives up after the deadline (error word
-// set) instead of waiting forever.
-__device__ __forceinline__ void grid_barrier(unsigned int* word, unsigned long long deadline, int* err)
+// were.  Thread 0 of each CTA keeps the bit it expects before its next arrival
+// (read once at kernel start: it cannot flip before this CTA arrives), so an
+// arrival is a fire-and-forget release reduction and only the poll waits.  The
+// poll acquires at GPU scope, so writes before the barrier are visible after
+// it.  Gives up after the deadline (error word set) instead of waiting forever.
+struct GridBar {
+    unsigned int* word;
+    unsigned int phase;  // bit 31 of the word before this CTA's next arrival (thread 0)
+};
+
+__device__ __forceinline__ GridBar grid_bar_open(unsigned int* word)
+{
+    GridBar b{word, 0u};
+    if (threadIdx.x == 0) {
+        unsigned int cur;
+        asm volatile("ld.relaxed.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(word) : "memory");
+        b.phase = cur & 0x80000000u;
+    }
+    return b;
+}
+
+__device__ __forceinline__ void grid_barrier(GridBar& b, unsigned long long deadline, int* err)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
         const unsigned int add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
-        unsigned int old, cur;
-        asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(word), "r"(add) : "memory");
+        asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(b.word), "r"(add) : "memory");
+        unsigned int cur;
         while (true) {
-            asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(word) : "memory");
-            if ((old ^ cur) & 0x80000000u) break;
+            asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(b.word) : "memory");
+            if ((cur ^ b.phase) & 0x80000000u) break;
             if (layer_ns() > deadline) {
                 atomicExch(err, 2);
                 break;
             }
-            __nanosleep(64);
         }
+        b.phase ^= 0x80000000u;
     }
     __syncthreads();
 }
@@ -205,7 +223,7 @@ __device__ __forceinline__ float lds32(uint32_t smem)
 
 template <int MT, int R, typename RowsOf, typename VecsOf, typename Finish, typename Hook = NoHook>
 __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per_lane, int nch, const float4* xs,
-                                                 const float* corr, unsigned char* ring, RowsOf rows_of,
+                                                 const void* corr, unsigned char* ring, RowsOf rows_of,
                                                  VecsOf vecs_of, Finish finish, Hook hook = Hook())
 {
     if (nj <= 0) {
@@ -263,8 +281,12 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
     float tot[2][MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
+    // staged vectors: one vector, digit planes (192 units of 16 bytes per step, a float2 per chunk);
+    // several vectors, float slots (256 units per step, a float per chunk)
+    constexpr int kXStep = MT == 1 ? kDigitPlanes * 32 : 256;
     const float4* xrow = xs;
-    const float* crow = corr + lane;
+    const float* crow = static_cast<const float*>(corr) + lane;
+    const float2* crow2 = static_cast<const float2*>(corr) + lane;
     const int S = nj * per_lane;
 #pragma unroll 1
     for (int s = 0; s < S; ++s) {
@@ -273,25 +295,32 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
         if (whole || lane + 32 * cci < nch) {
             const uint4 w0 = lds128(csl), w1 = lds128(csl + 512);
             const float s0 = lds32(csl + sc_off), s1 = lds32(csl + sc_off + 128);
-            float2 acc[2][MT];
-            chunk_pair_vectors<MT>(w0, w1, xrow, v, lane, acc);
+            if constexpr (MT == 1) {
+                chunk_pair_digits(w0, w1, reinterpret_cast<const uint4*>(xrow) + v.x4[0] + lane, crow2[v.cr[0]], s0,
+                                  s1, tot[0][0], tot[1][0]);
+            } else {
+                float2 acc[2][MT];
+                chunk_pair_vectors<MT>(w0, w1, xrow, v, lane, acc);
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
-                if (t < v.m) {
-                    const float cr = crow[v.cr[t]];
-                    tot[0][t] = chunk_finish(acc[0][t], cr, s0, tot[0][t]);
-                    tot[1][t] = chunk_finish(acc[1][t], cr, s1, tot[1][t]);
+                for (int t = 0; t < MT; ++t) {
+                    if (t < v.m) {
+                        const float cr = crow[v.cr[t]];
+                        tot[0][t] = chunk_finish(acc[0][t], cr, s0, tot[0][t]);
+                        tot[1][t] = chunk_finish(acc[1][t], cr, s1, tot[1][t]);
+                    }
                 }
             }
         }
         csl += kSlotBytes;
         if (csl == ring_end) csl = ring_lane;
-        xrow += 256;
+        xrow += kXStep;
         crow += 32;
+        crow2 += 32;
         if (++cci == per_lane) {
             cci = 0;
             xrow = xs;
-            crow = corr + lane;
+            crow = static_cast<const float*>(corr) + lane;
+            crow2 = static_cast<const float2*>(corr) + lane;
             finish(j0 + cj * js, v, tot);
 #pragma unroll
             for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
@@ -363,9 +392,9 @@ __host__ __device__ inline LayerSmem layer_smem(int T, int H, int F, int E, int 
     s.nh = out_rows ? k + 1 : MT;
     size_t off = 0;
     s.x_off = off;
-    off += align_up(stage_smem_bytes(H, s.nx), 16);
+    off += align_up(MT == 1 ? digit_smem_bytes(H, s.nx) : stage_smem_bytes(H, s.nx), 16);
     s.h_off = off;
-    off += align_up(stage_smem_bytes(F, s.nh), 16);
+    off += align_up(MT == 1 ? digit_smem_bytes(F, s.nh) : stage_smem_bytes(F, s.nh), 16);
     s.u_off = off;
     {
         const size_t P = (size_t)T * k;
@@ -752,11 +781,10 @@ __device__ __forceinline__ unsigned int* launch_barrier_word()
 }
 
 // Partial router scores of one piece: chunks c = lane + 32 p of router row e
-// (32 fp32 weights each) against the nt staged activation vectors; the warp's
-// sums go to logit_part[p][t][e].
-template <int NT>
-__device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, int nt, const StageGeom& g,
-                                             const float4* xs)
+// (32 fp32 weights each) against the nt tokens' activations, read in fp32 from
+// global memory (L2); the warp's sums go to logit_part[p][t][e].
+template <int NT, bool kBf16>
+__device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, int nt, const StageGeom& g)
 {
     const int lane = threadIdx.x & 31;
     const int c = lane + 32 * p;
@@ -772,14 +800,14 @@ __device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, i
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             if (t < nt) {
-                const float4* xr = xs + (size_t)t * g.f4 + p * 256;
+                const char* xr = static_cast<const char*>(a.x) + (size_t)t * a.H * (kBf16 ? 2 : 4);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const float4 xv = xr[j * 32 + (lane ^ j)];  // swapped pairs (x1, x0, x3, x2)
-                    acc[t] = fmaf(wv[j].x, xv.y, acc[t]);
-                    acc[t] = fmaf(wv[j].y, xv.x, acc[t]);
-                    acc[t] = fmaf(wv[j].z, xv.w, acc[t]);
-                    acc[t] = fmaf(wv[j].w, xv.z, acc[t]);
+                    const float4 xv = load_act4<kBf16>(xr, c * kChunkK + 4 * j);
+                    acc[t] = fmaf(wv[j].x, xv.x, acc[t]);
+                    acc[t] = fmaf(wv[j].y, xv.y, acc[t]);
+                    acc[t] = fmaf(wv[j].z, xv.z, acc[t]);
+                    acc[t] = fmaf(wv[j].w, xv.w, acc[t]);
                 }
             }
         }
@@ -814,18 +842,22 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
-    float* xcorr = reinterpret_cast<float*>(lsm + ls.x_off + (size_t)ls.nx * gH.f4 * 16);
+    // staged vectors: digit planes for one-vector groups, float slots otherwise (16-byte units per vector)
+    const int xvs = MT == 1 ? digit_vec_units(H) : gH.f4;
+    const int hvs = MT == 1 ? digit_vec_units(F) : gF.f4;
+    unsigned char* xcorr = lsm + ls.x_off + (size_t)ls.nx * xvs * 16;
     float4* hs = reinterpret_cast<float4*>(lsm + ls.h_off);
-    float* hcorr = reinterpret_cast<float*>(lsm + ls.h_off + (size_t)ls.nh * gF.f4 * 16);
+    unsigned char* hcorr = lsm + ls.h_off + (size_t)ls.nh * hvs * 16;
     const UnionSmem u = union_smem(lsm, ls);
     float* ypart = reinterpret_cast<float*>(lsm + ls.y_off);
     unsigned char* ring = lsm + ls.ring + (size_t)(threadIdx.x >> 5) * P_GU * kSlotBytes;  // this warp's ring
 
-    unsigned int* bar = launch_barrier_word();
-    if (!bar) {  // not a cooperative launch: nothing can be synchronised (same answer in every CTA)
+    unsigned int* bar_word = launch_barrier_word();
+    if (!bar_word) {  // not a cooperative launch: nothing can be synchronised (same answer in every CTA)
         if (blockIdx.x == 0 && threadIdx.x == 0) *a.err = 3;
         return;
     }
+    GridBar bar = grid_bar_open(bar_word);
     const unsigned long long deadline = layer_ns() + a.wait_ns;
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.err = 0;
     stamp(a, 0);
@@ -833,11 +865,19 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int n_sg = (T + MT - 1) / MT;  // shared-expert groups
 
     // activations / SwiGLU outputs into shared memory: vector t = row row0 + t (or tbl[t] / tdiv)
+    auto stage_vecs = [&](const void* src, int bf16, int K, int n, int row0, const int* tbl, int tdiv, float4* dst,
+                          unsigned char* dcorr, int tid, int nthr) {
+        if constexpr (MT == 1)
+            stage_rows_digits(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
+                              reinterpret_cast<float2*>(dcorr), tid, nthr);
+        else
+            stage_rows(src, bf16, K, n, row0, tbl, tdiv, dst, reinterpret_cast<float*>(dcorr), tid, nthr);
+    };
     auto stage_x = [&](int n, int row0, const int* tbl = nullptr, int tdiv = 1) {
-        stage_rows(a.x, kBf16 ? 1 : 0, H, n, row0, tbl, tdiv, xs, xcorr, (int)threadIdx.x, kLayerThreads);
+        stage_vecs(a.x, kBf16 ? 1 : 0, H, n, row0, tbl, tdiv, xs, xcorr, (int)threadIdx.x, kLayerThreads);
     };
     auto stage_h = [&](int n, int row0) {
-        stage_rows(a.h, 0, F, n, row0, nullptr, 1, hs, hcorr, (int)threadIdx.x, kLayerThreads);
+        stage_vecs(a.h, 0, F, n, row0, nullptr, 1, hs, hcorr, (int)threadIdx.x, kLayerThreads);
     };
 
     // gate/up item finisher: h[pos_t, n] = silu(gate) * up for the group's vectors
@@ -845,8 +885,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
             if (t < v.m) {
-                const float gv = warp_sum(tot[0][t]);
-                const float uv = warp_sum(tot[1][t]);
+                const float gu = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: gate, lane 16: up
+                const float gv = gu;
+                const float uv = __shfl_sync(0xFFFFFFFFu, gu, 16);
                 const int pos = pos0 + t;
                 if (lane == 0 && COLI_IN_BOUNDS(pos >= 0 && pos < P + T && n >= 0 && n < F, a.err))
                     a.h[(size_t)pos * F + n] = gv / (1.0f + expf(-gv)) * uv;
@@ -864,7 +905,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         auto router_pieces = [&]() {
             const int total = E * nrp;
             for (int i = blockIdx.x + gridDim.x * warp; i < total; i += gridDim.x * kLayerWarps)
-                router_piece<MT>(a, i / nrp, i % nrp, T, gH, xs);
+                router_piece<MT, kBf16>(a, i / nrp, i % nrp, T, gH);
         };
         auto stage_all = [&]() {
             stage_x(T, 0);
@@ -899,7 +940,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     const int vi = all_x ? t0 + t : t;
-                    v.x4[t] = vi * gH.f4;
+                    v.x4[t] = vi * xvs;
                     v.cr[t] = vi * gH.nch;
                 }
             };
@@ -1002,8 +1043,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 if (lane == 0) reinterpret_cast<int*>(u.tmp)[0] = n_kept;
                 stamp(a, 12);
             } else {
-                stage_rows(a.h, 0, F, 1, P, nullptr, 1, hs + (size_t)k * gF.f4, hcorr + (size_t)k * gF.nch,
-                           (int)threadIdx.x - 32, kLayerThreads - 32);
+                stage_vecs(a.h, 0, F, 1, P, nullptr, 1, hs + (size_t)k * hvs,
+                           hcorr + (size_t)k * gF.nch * (MT == 1 ? 8 : 4), (int)threadIdx.x - 32, kLayerThreads - 32);
                 stamp(a, 13, 32);
             }
             __syncthreads();
@@ -1020,16 +1061,13 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.m = 1;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    v.x4[t] = k * gF.f4;
+                    v.x4[t] = k * hvs;
                     v.cr[t] = k * gF.nch;
                 }
             };
             auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
-                const float y0 = warp_sum(tot[0][0]), y1 = warp_sum(tot[1][0]);
-                if (lane == 0) {
-                    ypart[(2 * j) * S1 + k] = y0;
-                    ypart[(2 * j + 1) * S1 + k] = y1;
-                }
+                const float y = warp_sum2(tot[0][0], tot[1][0]);  // lane 0: row 2 j, lane 16: row 2 j + 1
+                if ((lane & 15) == 0) ypart[(2 * j + (lane >> 4)) * S1 + k] = y;
             };
             const int first = warp;
             const int nj = first < npr ? (npr - first + kLayerWarps - 1) / kLayerWarps : 0;
@@ -1043,8 +1081,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int total = n_kept * F;
         const int lo = (int)((long long)total * blockIdx.x / gridDim.x);
         const int hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
+        const FastDiv div_f(F, total);
         auto rows_of = [&](int j, RowPair& r) {
-            const int g = j / F;
+            const int g = div_f(j);
             int e = u.gexp[g];
             if (!COLI_IN_BOUNDS(e >= 0 && e < E, a.err)) e = 0;
             const size_t row = (size_t)e * F + (j - g * F);
@@ -1062,7 +1101,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             }
         };
         auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
-            const int g = j / F;
+            const int g = div_f(j);
             gateup_finish(j - g * F, g, false, v, tot);
         };
         const int first = lo + warp;
@@ -1174,7 +1213,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.m = m;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    v.x4[t] = t * gF.f4;
+                    v.x4[t] = t * hvs;
                     v.cr[t] = t * gF.nch;
                 }
             };
@@ -1183,12 +1222,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     if (t < v.m) {
-                        const float y0 = warp_sum(tot[0][t]), y1 = warp_sum(tot[1][t]);
-                        if (lane == 0) {
-                            float* yr = a.y + (size_t)(P + t0 + t) * H + n;
-                            yr[0] = y0;
-                            yr[1] = y1;
-                        }
+                        const float y = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: row n, lane 16: row n + 1
+                        if ((lane & 15) == 0) a.y[(size_t)(P + t0 + t) * H + n + (lane >> 4)] = y;
                     }
                 }
             };
@@ -1233,7 +1268,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     const int vi = all_x ? (t < v.m ? u.perm[p0 + t] / k : 0) : t;
-                    v.x4[t] = vi * gH.f4;
+                    v.x4[t] = vi * xvs;
                     v.cr[t] = vi * gH.nch;
                 }
             };
@@ -1257,8 +1292,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int S = S1;
         // item j = (group g = j / npr: the g-th kept expert in ascending order, row pair)
         const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
+        const FastDiv div_pr(npr, (long long)npr * n_kept);
         auto rows_of = [&](int j, RowPair& r) {
-            const int slot = j / npr, pr = pr_lo + (j - slot * npr);
+            const int slot = div_pr(j), pr = pr_lo + (j - slot * npr);
             int e = u.gexp[slot];
             if (!COLI_IN_BOUNDS(e >= 0 && e < E && 2 * pr + 1 < H, a.err)) e = 0;
             const size_t row = (size_t)e * H + 2 * pr;
@@ -1268,21 +1304,18 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             r.s1 = r.s0 + F / kGroup;
         };
         auto vecs_of = [&](int j, VecSet<MT>& v) {
-            const int slot = j / npr;
+            const int slot = div_pr(j);
             v.m = 1;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-                v.x4[t] = slot * gF.f4;
+                v.x4[t] = slot * hvs;
                 v.cr[t] = slot * gF.nch;
             }
         };
         auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
-            const int slot = j / npr, pl = j - slot * npr;
-            const float y0 = warp_sum(tot[0][0]), y1 = warp_sum(tot[1][0]);
-            if (lane == 0) {
-                ypart[(2 * pl) * S + slot] = y0;
-                ypart[(2 * pl + 1) * S + slot] = y1;
-            }
+            const int slot = div_pr(j), pl = j - slot * npr;
+            const float y = warp_sum2(tot[0][0], tot[1][0]);  // lane 0: row 2 pl, lane 16: row 2 pl + 1
+            if ((lane & 15) == 0) ypart[(2 * pl + (lane >> 4)) * S + slot] = y;
         };
         auto hook = [&]() {
             grid_barrier(bar, deadline, a.err);
@@ -1341,7 +1374,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.m = m;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    v.x4[t] = t * gF.f4;
+                    v.x4[t] = t * hvs;
                     v.cr[t] = t * gF.nch;
                 }
             };
@@ -1350,12 +1383,10 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     if (t < v.m) {
-                        const float y0 = warp_sum(tot[0][t]), y1 = warp_sum(tot[1][t]);
-                        if (lane == 0 && COLI_IN_BOUNDS(p0 + t < P && n + 1 < H, a.err)) {
+                        const float y = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: row n, lane 16: row n + 1
+                        if ((lane & 15) == 0 && COLI_IN_BOUNDS(p0 + t < P && n + 1 < H, a.err)) {
                             const float wt = u.w[u.perm[p0 + t]];
-                            float* yr = a.y + (size_t)(p0 + t) * H + n;
-                            yr[0] = wt * y0;
-                            yr[1] = wt * y1;
+                            a.y[(size_t)(p0 + t) * H + n + (lane >> 4)] = wt * y;
                         }
                     }
                 }
