@@ -375,43 +375,6 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
     }
 }
 
-// Row-pair products of one chunk against a digit-staged vector: acc[row] gets
-// 2^(e - 21)-scaled exact integer sums (see above).  xd: this lane's plane 0 of
-// the chunk (planes 32 uint4 apart); c: the chunk's (scale, corr).
-__device__ __forceinline__ void chunk_pair_digits(const uint4& w0, const uint4& w1, const uint4* xd, float2 c,
-                                                  float s0, float s1, float& tot0, float& tot1)
-{
-    uint32_t al[4], ah[4], bl[4], bh[4];  // each word decoded once, used by the three digit planes
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t a = q == 0 ? w0.x : q == 1 ? w0.y : q == 2 ? w0.z : w0.w;
-        const uint32_t b = q == 0 ? w1.x : q == 1 ? w1.y : q == 2 ? w1.z : w1.w;
-        al[q] = nib_lo_u8(a);
-        ah[q] = nib_hi_u8(a);
-        bl[q] = nib_lo_u8(b);
-        bh[q] = nib_hi_u8(b);
-    }
-    int a0[3] = {0, 0, 0}, a1[3] = {0, 0, 0};
-#pragma unroll
-    for (int d = 0; d < 3; ++d) {
-        const uint4 xl = xd[(2 * d) * 32], xh = xd[(2 * d + 1) * 32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t l = q == 0 ? xl.x : q == 1 ? xl.y : q == 2 ? xl.z : xl.w;
-            const uint32_t h = q == 0 ? xh.x : q == 1 ? xh.y : q == 2 ? xh.z : xh.w;
-            a0[d] = dp4a_us(al[q], l, a0[d]);
-            a0[d] = dp4a_us(ah[q], h, a0[d]);
-            a1[d] = dp4a_us(bl[q], l, a1[d]);
-            a1[d] = dp4a_us(bh[q], h, a1[d]);
-        }
-    }
-    const uint32_t corr = (uint32_t)__float_as_int(c.y);
-    const uint32_t D0 = ((uint32_t)a0[0] * 128u + (uint32_t)a0[1]) * 128u + (uint32_t)a0[2] - corr;
-    const uint32_t D1 = ((uint32_t)a1[0] * 128u + (uint32_t)a1[1]) * 128u + (uint32_t)a1[2] - corr;
-    tot0 = fmaf(s0 * c.x, (float)(int)D0, tot0);
-    tot1 = fmaf(s1 * c.x, (float)(int)D1, tot1);
-}
-
 // The same with every thread of the block.
 template <typename Load4>
 __device__ __forceinline__ void stage_vectors_fn(int n, Load4 load, const StageGeom& g, float4* xs, float* corr)

@@ -44,9 +44,8 @@
 
 namespace coli {
 
-// Threads per block: 16 warps for one-token groups, 12 for four-token groups
-// (whose multiply-adds over four activation vectors need more registers).
-__host__ __device__ constexpr int layer_threads(int MT) { return MT == 1 ? 512 : 384; }
+// Threads per block: 16 warps (one CTA per SM, at most 128 registers a thread).
+__host__ __device__ constexpr int layer_threads(int) { return 512; }
 constexpr int kLayerMaxT = 64;      // tokens (64-bit token masks in the union)
 constexpr unsigned long long kBarrierNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
@@ -116,46 +115,58 @@ struct RowPair {
     const float* s1;
 };
 
-// The staged vectors (offsets of their float4 slots, and of their chunk
-// corrections) that one item multiplies its rows with.
+// The staged vectors that one item multiplies its rows with (indices into the
+// staged set: vector i's digit planes start i * vstride 16-byte units in, its
+// per-chunk (scale, corr) entries i * nch entries in).
 template <int MT>
 struct VecSet {
-    int m;         // vectors used (<= MT)
-    int x4[MT];    // float4 slot offset of vector t
-    int cr[MT];    // correction offset of vector t
+    int m;       // vectors used (<= MT)
+    int vi[MT];  // staged-vector index of vector t
 };
 
-// One 16-byte chunk of both rows against up to MT staged vectors: each packed
-// word of each row is decoded once and applied to every vector.
-// xrow = the staged slots of this lane's chunk row block; off = swizzle offsets.
+// One 16-byte chunk of both rows against up to MT digit-staged vectors (see
+// coli_int4.cuh): each word of each row is decoded once into biased bytes and
+// applied to every vector with dp4a.  xd = this lane's plane 0 of the chunk in
+// vector 0's frame; cc = this lane's chunk entry in vector 0's frame.
 template <int MT>
-__device__ __forceinline__ void chunk_pair_vectors(const uint4& w0, const uint4& w1, const float4* xrow,
-                                                   const VecSet<MT>& v, int lane, float2 (&acc)[2][MT])
+__device__ __forceinline__ void chunk_pair_digit_vectors(const uint4& w0, const uint4& w1, const uint4* xd,
+                                                         const float2* cc, const VecSet<MT>& v, int vstride, int nch,
+                                                         float s0, float s1, float (&tot)[2][MT])
 {
-#pragma unroll
-    for (int t = 0; t < MT; ++t) acc[0][t] = acc[1][t] = make_float2(0.f, 0.f);
+    uint32_t al[4], ah[4], bl[4], bh[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint32_t a = q == 0 ? w0.x : q == 1 ? w0.y : q == 2 ? w0.z : w0.w;
         const uint32_t b = q == 0 ? w1.x : q == 1 ? w1.y : q == 2 ? w1.z : w1.w;
-        const float2 a0 = nib_pair(a << 15), a1 = nib_pair(a << 7), a2 = nib_pair(a >> 1), a3 = nib_pair(a >> 9);
-        const float2 b0 = nib_pair(b << 15), b1 = nib_pair(b << 7), b2 = nib_pair(b >> 1), b3 = nib_pair(b >> 9);
+        al[q] = nib_lo_u8(a);
+        ah[q] = nib_hi_u8(a);
+        bl[q] = nib_lo_u8(b);
+        bh[q] = nib_hi_u8(b);
+    }
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            if (t < v.m) {
-                const float4 xlo = xrow[v.x4[t] + (2 * q) * 32 + (lane ^ (2 * q))];
-                const float4 xhi = xrow[v.x4[t] + (2 * q + 1) * 32 + (lane ^ (2 * q + 1))];
-                const float2 p0 = make_float2(xlo.x, xlo.y), p1 = make_float2(xlo.z, xlo.w);
-                const float2 p2 = make_float2(xhi.x, xhi.y), p3 = make_float2(xhi.z, xhi.w);
-                acc[0][t] = __ffma2_rn(a0, p0, acc[0][t]);
-                acc[1][t] = __ffma2_rn(b0, p0, acc[1][t]);
-                acc[0][t] = __ffma2_rn(a1, p1, acc[0][t]);
-                acc[1][t] = __ffma2_rn(b1, p1, acc[1][t]);
-                acc[0][t] = __ffma2_rn(a2, p2, acc[0][t]);
-                acc[1][t] = __ffma2_rn(b2, p2, acc[1][t]);
-                acc[0][t] = __ffma2_rn(a3, p3, acc[0][t]);
-                acc[1][t] = __ffma2_rn(b3, p3, acc[1][t]);
+    for (int t = 0; t < MT; ++t) {
+        if (t < v.m) {
+            const uint4* x = xd + v.vi[t] * vstride;
+            int a0[3] = {0, 0, 0}, a1[3] = {0, 0, 0};
+#pragma unroll
+            for (int d = 0; d < 3; ++d) {
+                const uint4 xl = x[(2 * d) * 32], xh = x[(2 * d + 1) * 32];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t l = q == 0 ? xl.x : q == 1 ? xl.y : q == 2 ? xl.z : xl.w;
+                    const uint32_t h = q == 0 ? xh.x : q == 1 ? xh.y : q == 2 ? xh.z : xh.w;
+                    a0[d] = dp4a_us(al[q], l, a0[d]);
+                    a0[d] = dp4a_us(ah[q], h, a0[d]);
+                    a1[d] = dp4a_us(bl[q], l, a1[d]);
+                    a1[d] = dp4a_us(bh[q], h, a1[d]);
+                }
             }
+            const float2 c = cc[v.vi[t] * nch];
+            const uint32_t corr = (uint32_t)__float_as_int(c.y);
+            const uint32_t D0 = ((uint32_t)a0[0] * 128u + (uint32_t)a0[1]) * 128u + (uint32_t)a0[2] - corr;
+            const uint32_t D1 = ((uint32_t)a1[0] * 128u + (uint32_t)a1[1]) * 128u + (uint32_t)a1[2] - corr;
+            tot[0][t] = fmaf(s0 * c.x, (float)(int)D0, tot[0][t]);
+            tot[1][t] = fmaf(s1 * c.x, (float)(int)D1, tot[1][t]);
         }
     }
 }
@@ -281,12 +292,11 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
     float tot[2][MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
-    // staged vectors: one vector, digit planes (192 units of 16 bytes per step, a float2 per chunk);
-    // several vectors, float slots (256 units per step, a float per chunk)
-    constexpr int kXStep = MT == 1 ? kDigitPlanes * 32 : 256;
-    const float4* xrow = xs;
-    const float* crow = static_cast<const float*>(corr) + lane;
-    const float2* crow2 = static_cast<const float2*>(corr) + lane;
+    // staged vectors: digit planes, 6 x 32 units of 16 bytes per chunk step; a float2 entry per chunk
+    constexpr int kXStep = kDigitPlanes * 32;
+    const int vstride = per_lane * kXStep;  // 16-byte units per staged vector
+    const uint4* xrow = reinterpret_cast<const uint4*>(xs) + lane;
+    const float2* crow = static_cast<const float2*>(corr) + lane;
     const int S = nj * per_lane;
 #pragma unroll 1
     for (int s = 0; s < S; ++s) {
@@ -295,32 +305,16 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
         if (whole || lane + 32 * cci < nch) {
             const uint4 w0 = lds128(csl), w1 = lds128(csl + 512);
             const float s0 = lds32(csl + sc_off), s1 = lds32(csl + sc_off + 128);
-            if constexpr (MT == 1) {
-                chunk_pair_digits(w0, w1, reinterpret_cast<const uint4*>(xrow) + v.x4[0] + lane, crow2[v.cr[0]], s0,
-                                  s1, tot[0][0], tot[1][0]);
-            } else {
-                float2 acc[2][MT];
-                chunk_pair_vectors<MT>(w0, w1, xrow, v, lane, acc);
-#pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    if (t < v.m) {
-                        const float cr = crow[v.cr[t]];
-                        tot[0][t] = chunk_finish(acc[0][t], cr, s0, tot[0][t]);
-                        tot[1][t] = chunk_finish(acc[1][t], cr, s1, tot[1][t]);
-                    }
-                }
-            }
+            chunk_pair_digit_vectors<MT>(w0, w1, xrow, crow, v, vstride, nch, s0, s1, tot);
         }
         csl += kSlotBytes;
         if (csl == ring_end) csl = ring_lane;
         xrow += kXStep;
         crow += 32;
-        crow2 += 32;
         if (++cci == per_lane) {
             cci = 0;
-            xrow = xs;
-            crow = static_cast<const float*>(corr) + lane;
-            crow2 = static_cast<const float2*>(corr) + lane;
+            xrow = reinterpret_cast<const uint4*>(xs) + lane;
+            crow = static_cast<const float2*>(corr) + lane;
             finish(j0 + cj * js, v, tot);
 #pragma unroll
             for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
@@ -392,9 +386,9 @@ __host__ __device__ inline LayerSmem layer_smem(int T, int H, int F, int E, int 
     s.nh = out_rows ? k + 1 : MT;
     size_t off = 0;
     s.x_off = off;
-    off += align_up(MT == 1 ? digit_smem_bytes(H, s.nx) : stage_smem_bytes(H, s.nx), 16);
+    off += align_up(digit_smem_bytes(H, s.nx), 16);
     s.h_off = off;
-    off += align_up(MT == 1 ? digit_smem_bytes(F, s.nh) : stage_smem_bytes(F, s.nh), 16);
+    off += align_up(digit_smem_bytes(F, s.nh), 16);
     s.u_off = off;
     {
         const size_t P = (size_t)T * k;
@@ -842,9 +836,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
-    // staged vectors: digit planes for one-vector groups, float slots otherwise (16-byte units per vector)
-    const int xvs = MT == 1 ? digit_vec_units(H) : gH.f4;
-    const int hvs = MT == 1 ? digit_vec_units(F) : gF.f4;
+    // staged vectors as digit planes (16-byte units per vector)
+    const int xvs = digit_vec_units(H);
+    const int hvs = digit_vec_units(F);
     unsigned char* xcorr = lsm + ls.x_off + (size_t)ls.nx * xvs * 16;
     float4* hs = reinterpret_cast<float4*>(lsm + ls.h_off);
     unsigned char* hcorr = lsm + ls.h_off + (size_t)ls.nh * hvs * 16;
@@ -867,11 +861,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     // activations / SwiGLU outputs into shared memory: vector t = row row0 + t (or tbl[t] / tdiv)
     auto stage_vecs = [&](const void* src, int bf16, int K, int n, int row0, const int* tbl, int tdiv, float4* dst,
                           unsigned char* dcorr, int tid, int nthr) {
-        if constexpr (MT == 1)
-            stage_rows_digits(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
-                              reinterpret_cast<float2*>(dcorr), tid, nthr);
-        else
-            stage_rows(src, bf16, K, n, row0, tbl, tdiv, dst, reinterpret_cast<float*>(dcorr), tid, nthr);
+        stage_rows_digits(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
+                          reinterpret_cast<float2*>(dcorr), tid, nthr);
     };
     auto stage_x = [&](int n, int row0, const int* tbl = nullptr, int tdiv = 1) {
         stage_vecs(a.x, kBf16 ? 1 : 0, H, n, row0, tbl, tdiv, xs, xcorr, (int)threadIdx.x, kLayerThreads);
@@ -940,8 +931,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     const int vi = all_x ? t0 + t : t;
-                    v.x4[t] = vi * xvs;
-                    v.cr[t] = vi * gH.nch;
+                    v.vi[t] = vi;
                 }
             };
             auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
@@ -1044,7 +1034,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 stamp(a, 12);
             } else {
                 stage_vecs(a.h, 0, F, 1, P, nullptr, 1, hs + (size_t)k * hvs,
-                           hcorr + (size_t)k * gF.nch * (MT == 1 ? 8 : 4), (int)threadIdx.x - 32, kLayerThreads - 32);
+                           hcorr + (size_t)k * gF.nch * 8, (int)threadIdx.x - 32, kLayerThreads - 32);
                 stamp(a, 13, 32);
             }
             __syncthreads();
@@ -1061,8 +1051,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.m = 1;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    v.x4[t] = k * hvs;
-                    v.cr[t] = k * gF.nch;
+                    v.vi[t] = k;
                 }
             };
             auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
@@ -1096,8 +1085,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             v.m = 1;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-                v.x4[t] = 0;
-                v.cr[t] = 0;
+                v.vi[t] = 0;
             }
         };
         auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
@@ -1213,8 +1201,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.m = m;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    v.x4[t] = t * hvs;
-                    v.cr[t] = t * gF.nch;
+                    v.vi[t] = t;
                 }
             };
             auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
@@ -1268,8 +1255,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     const int vi = all_x ? (t < v.m ? u.perm[p0 + t] / k : 0) : t;
-                    v.x4[t] = vi * xvs;
-                    v.cr[t] = vi * gH.nch;
+                    v.vi[t] = vi;
                 }
             };
             auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
@@ -1308,8 +1294,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             v.m = 1;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-                v.x4[t] = slot * hvs;
-                v.cr[t] = slot * gF.nch;
+                v.vi[t] = slot;
             }
         };
         auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
@@ -1374,8 +1359,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.m = m;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    v.x4[t] = t * hvs;
-                    v.cr[t] = t * gF.nch;
+                    v.vi[t] = t;
                 }
             };
             auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
