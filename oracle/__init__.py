@@ -46,6 +46,11 @@ def lib():
         L.coli_oracle_moe_layer_top_p.restype = ctypes.c_int
         L.coli_oracle_moe_layer_top_p.argtypes = [_ptr, _i64, _i64, _i64, _i64, _i64, _dbl, _dbl,
                                                   _ptr, _ptr] + [_ptr] * 6 + [_ptr, _ptr, _ptr]
+        L.coli_oracle_quant_i8.restype = ctypes.c_int
+        L.coli_oracle_quant_i8.argtypes = [_ptr, _i64, _ptr, _ptr]
+        L.coli_oracle_moe_layer_i8.restype = ctypes.c_int
+        L.coli_oracle_moe_layer_i8.argtypes = [_ptr, _i64, _i64, _i64, _i64, _i64, _dbl,
+                                               _ptr, _ptr] + [_ptr] * 6 + [_ptr, _ptr, _ptr]
         L.coli_oracle_threads.restype = ctypes.c_int
         L.coli_oracle_threads.argtypes = []
         _lib = L
@@ -217,4 +222,33 @@ def moe_layer(x, H, F, E, k, routed_scale, w_router, sel_bias, experts):
                                        _p(w_router), _p(sel_bias),
                                        *[ctypes.cast(t, ctypes.c_void_p) for t in tables],
                                        _p(idx), _p(w), _p(out)), "moe_layer")
+    return idx, w, out
+
+
+def quant_i8(x):
+    """Integer-activation codes of fp32 values x [..., n] (n a multiple of 32):
+    (codes int8 [..., n], scales fp32 [..., n / 32])."""
+    x = _c(x, np.float32)
+    n = x.shape[-1]
+    codes = np.empty(x.shape, np.int8)
+    scales = np.empty(x.shape[:-1] + (n // 32,), np.float32)
+    _check(lib().coli_oracle_quant_i8(_p(x), x.size, _p(codes), _p(scales)), "quant_i8")
+    return codes, scales
+
+
+def moe_layer_i8(x, H, F, E, k, routed_scale, w_router, sel_bias, experts):
+    """The layer with int8 activations into every expert product.  Returns
+    (idx, w, out [T,H] f64)."""
+    x = _c(widen(x), np.float64)
+    T = x.shape[0]
+    w_router = _c(w_router, np.float32); sel_bias = _c(sel_bias, np.float32)
+    keep, tables = _expert_tables(experts, E)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    out = np.empty((T, H), np.float64)
+    _check(lib().coli_oracle_moe_layer_i8(_p(x), T, H, F, E, k, float(routed_scale),
+                                          _p(w_router), _p(sel_bias),
+                                          *[ctypes.cast(t, ctypes.c_void_p) for t in tables],
+                                          _p(idx), _p(w), _p(out)), "moe_layer_i8")
+    del keep
     return idx, w, out

@@ -359,3 +359,127 @@ int coli_oracle_moe_layer_top_p(const double* x, int64_t T, int64_t H, int64_t F
     free(y);
     return 0;
 }
+
+/*
+ * Integer-activation variant ("Colibri 完全ガイド", section コア技術のハイライト,
+ * row 整数ドット積カーネル: int8 and packed-int4 integer products from u8 x s8
+ * pairs, so the activations are int8; the same page's environment table lists
+ * the IDOT switch).  The pages name the kernel but not its quantisation rule;
+ * this library reads it as symmetric int8 per block of 32 consecutive values:
+ *   m = max |x| over the block,  scale = m / 127,
+ *   code = rint(x * (127 / m))   (round half to even), in [-127, 127],
+ *   x_hat = code * scale;  an all-zero block has codes 0 and scale 0, and a
+ *   block holding inf or NaN has codes 0 and scale NaN.
+ * Every step is taken in fp32, the precision the kernel decides the codes in.
+ */
+#define COLI_ORACLE_I8_BLOCK 32
+
+int coli_oracle_quant_i8(const float* x, int64_t n, int8_t* code, float* scale)
+{
+    if (!x || !code || !scale || n < 0 || n % COLI_ORACLE_I8_BLOCK != 0) return -1;
+    for (int64_t b = 0; b < n / COLI_ORACLE_I8_BLOCK; ++b) {
+        const float* xb = x + b * COLI_ORACLE_I8_BLOCK;
+        int8_t* cb = code + b * COLI_ORACLE_I8_BLOCK;
+        float m = 0.0f;
+        int finite = 1;
+        for (int i = 0; i < COLI_ORACLE_I8_BLOCK; ++i) {
+            if (!isfinite(xb[i])) finite = 0;
+            else if (fabsf(xb[i]) > m) m = fabsf(xb[i]);
+        }
+        if (!finite || m == 0.0f) {
+            for (int i = 0; i < COLI_ORACLE_I8_BLOCK; ++i) cb[i] = 0;
+            scale[b] = finite ? 0.0f : NAN;
+            continue;
+        }
+        const float inv = 127.0f / m;
+        for (int i = 0; i < COLI_ORACLE_I8_BLOCK; ++i) {
+            float c = rintf(xb[i] * inv);
+            if (c > 127.0f) c = 127.0f;
+            if (c < -127.0f) c = -127.0f;
+            cb[i] = (int8_t)c;
+        }
+        scale[b] = m / 127.0f;
+    }
+    return 0;
+}
+
+/* x_hat of a vector of n values (fp32 x given as f64, widened exactly from fp32). */
+static int quant_i8_hat(const double* x, int64_t n, double* xh)
+{
+    if (n <= 0) return -1;
+    float* xf = (float*)malloc(sizeof(float) * (size_t)n);
+    int8_t* c = (int8_t*)malloc((size_t)n);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(n / COLI_ORACLE_I8_BLOCK + 1));
+    if (!xf || !c || !s) { free(xf); free(c); free(s); return -1; }
+    for (int64_t i = 0; i < n; ++i) xf[i] = (float)x[i];
+    int rc = coli_oracle_quant_i8(xf, n, c, s);
+    if (rc == 0)
+        for (int64_t i = 0; i < n; ++i) xh[i] = (double)c[i] * (double)s[i / COLI_ORACLE_I8_BLOCK];
+    free(xf); free(c); free(s);
+    return rc;
+}
+
+/*
+ * One expert with int8 activations: g = Wg x_hat, u = Wu x_hat,
+ * h = silu(g) * u (f64, rounded to fp32 before it is quantised, as the kernel
+ * holds it), y = Wd h_hat.
+ */
+static int expert_ffn_i8(const double* x, int64_t H, int64_t F,
+                         const uint8_t* gate_q, const float* gate_s, const uint8_t* up_q, const float* up_s,
+                         const uint8_t* down_q, const float* down_s, double* y)
+{
+    double* xh = (double*)malloc(sizeof(double) * (size_t)H);
+    double* g = (double*)malloc(sizeof(double) * (size_t)F);
+    double* u = (double*)malloc(sizeof(double) * (size_t)F);
+    double* a = (double*)malloc(sizeof(double) * (size_t)F);
+    double* ah = (double*)malloc(sizeof(double) * (size_t)F);
+    int rc = -1;
+    if (xh && g && u && a && ah && quant_i8_hat(x, H, xh) == 0) {
+        coli_oracle_matvec(gate_q, gate_s, F, H, xh, g);
+        coli_oracle_matvec(up_q, up_s, F, H, xh, u);
+        for (int64_t f = 0; f < F; ++f) a[f] = (double)(float)(g[f] * sigmoid(g[f]) * u[f]);
+        if (quant_i8_hat(a, F, ah) == 0) rc = coli_oracle_matvec(down_q, down_s, H, F, ah, y);
+    }
+    free(xh); free(g); free(u); free(a); free(ah);
+    return rc;
+}
+
+/*
+ * The layer with int8 activations in every expert: the route is the plain one
+ * (the router reads the activations as stored), out_t = sum_j w[t,j] *
+ * FFN8_{idx[t,j]}(x_t) + FFN8_E(x_t), FFN8 = expert_ffn_i8.
+ */
+int coli_oracle_moe_layer_i8(const double* x, int64_t T, int64_t H, int64_t F,
+                             int64_t E, int64_t k, double routed_scale,
+                             const float* w_router, const float* sel_bias,
+                             const uint8_t* const* gate_q, const float* const* gate_s,
+                             const uint8_t* const* up_q, const float* const* up_s,
+                             const uint8_t* const* down_q, const float* const* down_s,
+                             int32_t* topk_idx, double* topk_w, double* out)
+{
+    if (!x || !gate_q || !gate_s || !up_q || !up_s || !down_q || !down_s) return -1;
+    if (!topk_idx || !topk_w || !out) return -1;
+    if (H % COLI_ORACLE_I8_BLOCK != 0 || F % COLI_ORACLE_I8_BLOCK != 0) return -1;
+    int rc = coli_oracle_route(x, T, H, w_router, sel_bias, E, k, routed_scale, topk_idx, topk_w, NULL, NULL, NULL);
+    if (rc != 0) return rc;
+    double* y = (double*)malloc(sizeof(double) * (size_t)H);
+    if (!y) return -1;
+    for (int64_t t = 0; t < T; ++t) {
+        const double* xt = x + t * H;
+        double* ot = out + t * H;
+        for (int64_t n = 0; n < H; ++n) ot[n] = 0.0;
+        for (int64_t j = 0; j <= k; ++j) {
+            const int64_t e = j < k ? topk_idx[t * k + j] : E;
+            if (!gate_q[e] || !gate_s[e] || !up_q[e] || !up_s[e] || !down_q[e] || !down_s[e]) {
+                free(y);
+                return -1;
+            }
+            rc = expert_ffn_i8(xt, H, F, gate_q[e], gate_s[e], up_q[e], up_s[e], down_q[e], down_s[e], y);
+            if (rc != 0) { free(y); return rc; }
+            const double wj = j < k ? topk_w[t * k + j] : 1.0;
+            for (int64_t n = 0; n < H; ++n) ot[n] += wj * y[n];
+        }
+    }
+    free(y);
+    return 0;
+}

@@ -17,6 +17,9 @@
  *   - Expert FFN on int4 weights with one scale per group of 64 along K
  *     ("colibri: 744B MoE…", section はじめにとソースが語らないこと, "gs64 build";
  *      mcpfield "colibri" page, section コアアーキテクチャ, int4 experts).
+ *   - Integer-activation variant: int8 activations per block of 32 into the
+ *     expert products ("Colibri 完全ガイド", section コア技術のハイライト, row
+ *     整数ドット積カーネル).
  *   - Shared expert, always on, added with weight one
  *     ("Colibri 完全ガイド", same row; Korean page, section 프로젝트 설명, shared experts).
  *
@@ -104,6 +107,20 @@ int coli_oracle_moe_layer_top_p(const double* x, int64_t T, int64_t H, int64_t F
                                 const uint8_t* const* up_q, const float* const* up_s,
                                 const uint8_t* const* down_q, const float* const* down_s,
                                 int32_t* topk_idx, double* topk_w, double* out);
+
+/* Integer-activation variant (see coli_oracle.c): symmetric int8 codes of x
+ * [n] (n a multiple of 32), one fp32 scale per block of 32. */
+int coli_oracle_quant_i8(const float* x, int64_t n, int8_t* code, float* scale);
+
+/* The layer with int8 activations into every expert matmul (x before gate/up,
+ * h before down); the route reads the stored activations. */
+int coli_oracle_moe_layer_i8(const double* x, int64_t T, int64_t H, int64_t F,
+                             int64_t E, int64_t k, double routed_scale,
+                             const float* w_router, const float* sel_bias,
+                             const uint8_t* const* gate_q, const float* const* gate_s,
+                             const uint8_t* const* up_q, const float* const* up_s,
+                             const uint8_t* const* down_q, const float* const* down_s,
+                             int32_t* topk_idx, double* topk_w, double* out);
 
 #ifdef __cplusplus
 }
