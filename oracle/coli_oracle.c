@@ -11,6 +11,7 @@
  */
 #include "coli_oracle.h"
 
+#include <float.h>
 #include <math.h>
 #include <stddef.h>
 #include <stdlib.h>
@@ -368,8 +369,9 @@ int coli_oracle_moe_layer_top_p(const double* x, int64_t T, int64_t H, int64_t F
  * this library reads it as symmetric int8 per block of 32 consecutive values:
  *   m = max |x| over the block,  scale = m / 127,
  *   code = rint(x * (127 / m))   (round half to even), in [-127, 127],
- *   x_hat = code * scale;  an all-zero block has codes 0 and scale 0, and a
- *   block holding inf or NaN has codes 0 and scale NaN.
+ *   x_hat = code * scale;  an all-zero block (or one whose maximum is so small
+ *   that 127 / m overflows fp32) has codes 0 and scale 0, and a block holding
+ *   inf or NaN has codes 0 and scale NaN.
  * Every step is taken in fp32, the precision the kernel decides the codes in.
  */
 #define COLI_ORACLE_I8_BLOCK 32
@@ -392,6 +394,11 @@ int coli_oracle_quant_i8(const float* x, int64_t n, int8_t* code, float* scale)
             continue;
         }
         const float inv = 127.0f / m;
+        if (!(inv <= FLT_MAX)) { /* a maximum below 127 / FLT_MAX: the block is taken as zero */
+            for (int i = 0; i < COLI_ORACLE_I8_BLOCK; ++i) cb[i] = 0;
+            scale[b] = 0.0f;
+            continue;
+        }
         for (int i = 0; i < COLI_ORACLE_I8_BLOCK; ++i) {
             float c = rintf(xb[i] * inv);
             if (c > 127.0f) c = 127.0f;
