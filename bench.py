@@ -71,6 +71,8 @@ def parse(argv=None):
     ap.add_argument("--experts", type=int, default=0,
                     help="routed experts per layer (0 = the workload's; profiling: fewer, same per-call bytes)")
     ap.add_argument("--replays", type=int, default=0, help="timed replays of the K steps (0 = sized to ~0.3 s)")
+    ap.add_argument("--int8", action="store_true",
+                    help="also time the integer-activation variant of the chosen --config (always with no --config)")
     ap.add_argument("--top-p", type=float, default=0.0,
                     help="also time decode batch 1 with adaptive expert top-p (0 = the default 0.7 entry only "
                          "when all workloads run)")
@@ -327,9 +329,22 @@ class Resident:
         self.H, self.F, self.E = c.H, c.F, c.E
 
 
-def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sampler_index, top_p=0.0):
+def path_dtype(path, act_int8=False):
+    """Arithmetic the timed path computes in: the tensor-core prefill in bf16
+    operands with fp32 accumulation; the decode kernel in exact int32 products
+    of int4 weights and fixed-point (21-bit, or int8 for the variant)
+    activations, accumulated in fp32; the CUDA-core wide path in fp32."""
+    if path == "prefill":
+        return "bf16"
+    if path in ("single", "decode"):
+        return "int8xint4->int32/f32" if act_int8 else "int32/f32"
+    return "f32"
+
+
+def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sampler_index, top_p=0.0, act_int8=False):
     """Time one workload; returns the fields of its benchmark entry.  top_p > 0
-    runs the layer with adaptive expert top-p routing."""
+    runs the layer with adaptive expert top-p routing; act_int8 the
+    integer-activation variant (int8 activations per 32 values)."""
     hbm_peak, bf16_peak, bf16_sust, peak_kind = peaks
     routers, layers = [], []
     for l in range(N_LAYERS):
@@ -338,7 +353,7 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         b = res.bufs[l]
         layers.append(coli.Layer(c.H, c.F, c.E, c.k, c.routed_scale, torch.from_numpy(w_router).cuda(),
                                  torch.from_numpy(sel_bias).cuda(), b["gate_q"], b["gate_s"], b["up_q"],
-                                 b["up_s"], b["down_q"], b["down_s"], top_p=top_p))
+                                 b["up_s"], b["down_q"], b["down_s"], top_p=top_p, act_int8=act_int8))
     path = coli.moe_path(layers[0], c.T)
 
     # activation pool: G distinct (step, layer) batches, G a multiple of the layer count
@@ -482,8 +497,10 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         alg = roofline.get("alg_bytes_per_launch")
         roofline["traffic_over_alg"] = traffic / alg if alg else None
     expert_alg = float(np.mean((U + 1) * c.expert_bytes))  # selected experts' int4 + scales only
-    entry = {"workload": workload_desc(c) + (f", adaptive expert top-p {top_p}" if top_p else ""),
-             "tokens_per_call": c.T, "path": path, "value": value, "top_p": top_p,
+    entry = {"workload": workload_desc(c) + (f", adaptive expert top-p {top_p}" if top_p else "") +
+             (", int8 activations (integer-dot variant)" if act_int8 else ""),
+             "tokens_per_call": c.T, "path": path, "value": value, "top_p": top_p, "act_int8": bool(act_int8),
+             "dtype": path_dtype(path, act_int8),
              "unit": "tokens/s", "steps": steps, "timed_replays": R, "ms_per_step": ms_per_step,
              "ms_per_step_p10": percentile(ms_max, 10) / steps, "ms_per_step_p90": percentile(ms_max, 90) / steps,
              "roofline": roofline, "gpu_launches": steps * kernels_per_call(path, c.T, c.E),
@@ -572,6 +589,13 @@ def run_ours(args):
         entries[k] = measure_workload(args, torch, coli, cfg_of(k), res, seed, world, rank, peaks,
                                       torch.cuda.current_device())
         torch.cuda.empty_cache()
+    int8 = {}
+    if not args.config or args.int8:
+        # the integer-activation variant (int8 activations into the expert products)
+        for k in ([args.config] if args.config else [1, 2, 3]):
+            int8[k] = measure_workload(args, torch, coli, cfg_of(k), res, seed, world, rank, peaks,
+                                       torch.cuda.current_device(), act_int8=True)
+            torch.cuda.empty_cache()
     topp = None
     if not args.config or args.top_p:
         # decode batch 1 with the pages' --topp 0.7 knob: fewer expert bytes per token
@@ -589,14 +613,16 @@ def run_ours(args):
              "expert_alg_bytes_per_call": head["expert_alg_bytes_per_call"],
              "expert_frac_of_hbm_peak": head["expert_frac_of_hbm_peak"], "stage_ms": head["stage_ms"],
              "timing": "median of the timed replays of exactly K steps (CUDA events, max over ranks)"}
-    if len(cfgs) > 1 or topp is not None:
+    if len(cfgs) > 1 or topp is not None or int8:
         extra["per_workload"] = {cfg_of(k).name: entries[k] for k in cfgs[1:]}
         if topp is not None:
             extra["per_workload"][f"{cfg_of(1).name}-topp{topp['top_p']}"] = topp
+        for k, ent in int8.items():
+            extra["per_workload"][f"{cfg_of(k).name}-int8"] = ent
     line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": head["steps"],
             "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if head["path"] == "prefill" else "f32", "data": "synthetic",
+            "dtype": head["dtype"], "data": "synthetic",
             "config": config_block(c, head["graph_calls"], extra),
             "roofline": head["roofline"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"]}
     if "e2e" in head:

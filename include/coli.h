@@ -78,6 +78,7 @@ typedef struct {
     const float* up_s;     /* [E+1, F, H/64] */
     const float* down_s;   /* [E+1, H, F/64] */
     float top_p;           /* adaptive expert top-p: 0 (or >= 1) = plain top-k; see coli_moe_forward */
+    int act_int8;          /* 1: integer-activation variant (int8 activations per 32); 0: default; see coli_moe_forward */
 } coli_moe_layer;
 
 /*
@@ -148,8 +149,19 @@ COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
  * knob and its effect only.  The router is fp32.  Batches of up to 64 tokens
  * compute the experts in fp32 (bf16 x is widened exactly); larger batches run
  * them on the tensor cores with bf16 operands (weights q * scale, activations
- * and the SwiGLU output rounded to bf16) and fp32 accumulation.  out is written
- * as fp32 or bf16 (round to nearest even).
+ * and the SwiGLU output rounded to bf16) and fp32 accumulation.  In the
+ * 1-64-token kernel the activations enter the expert products as 21-bit fixed
+ * point per block of 32 values (power-of-two block scale; each value within
+ * 2^-21 of its block's largest magnitude) with exact integer products, an
+ * error of the same order as fp32 arithmetic.
+ * Integer-activation variant (layer->act_int8 = 1; "Colibri 完全ガイド", section
+ * コア技術のハイライト, row 整数ドット積カーネル, int8 activations times packed
+ * int4 weights): x before gate/up and h before down are quantised to
+ * symmetric int8 per block of 32 (scale max|v| / 127, codes rint(v * 127 /
+ * max|v|) in fp32) and multiplied exactly in integers; routing is unchanged.
+ * The quantisation rule is this library's reading.  Batches of up to 64 tokens
+ * only: a larger batch with act_int8 set returns COLI_ERR_UNSUPPORTED.  out is
+ * written as fp32 or bf16 (round to nearest even).
  * x [T, H] dtype xt; out [T, H] dtype ot; workspace of at least
  * coli_moe_workspace_size(layer, T) bytes, contents undefined on entry and on
  * exit apart from the status word (coli_moe_status_word_offset), not shared by

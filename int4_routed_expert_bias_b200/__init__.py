@@ -63,7 +63,8 @@ class _LayerStruct(ctypes.Structure):
                 ("routed_scale", ctypes.c_float),
                 ("w_router", _p), ("sel_bias", _p),
                 ("gate_q", _p), ("up_q", _p), ("down_q", _p),
-                ("gate_s", _p), ("up_s", _p), ("down_s", _p), ("top_p", ctypes.c_float)]
+                ("gate_s", _p), ("up_s", _p), ("down_s", _p), ("top_p", ctypes.c_float),
+                ("act_int8", ctypes.c_int)]
 
 
 def lib():
@@ -107,7 +108,7 @@ class Layer:
     """One MoE layer: device tensors in the library's layout (expert E = shared)."""
 
     def __init__(self, hidden, ffn, n_experts, top_k, routed_scale, w_router, sel_bias,
-                 gate_q, gate_s, up_q, up_s, down_q, down_s, group=64, top_p=0.0):
+                 gate_q, gate_s, up_q, up_s, down_q, down_s, group=64, top_p=0.0, act_int8=False):
         self.tensors = dict(w_router=w_router, sel_bias=sel_bias, gate_q=gate_q, gate_s=gate_s,
                             up_q=up_q, up_s=up_s, down_q=down_q, down_s=down_s)
         self.hidden, self.ffn, self.n_experts, self.top_k = hidden, ffn, n_experts, top_k
@@ -115,7 +116,7 @@ class Layer:
         self.struct = _LayerStruct(hidden, ffn, n_experts, top_k, group, routed_scale,
                                    *[_ptr(self.tensors[n]) for n in
                                      ("w_router", "sel_bias", "gate_q", "up_q", "down_q", "gate_s", "up_s",
-                                      "down_s")], float(top_p))
+                                      "down_s")], float(top_p), 1 if act_int8 else 0)
 
     @property
     def ref(self):

@@ -248,6 +248,7 @@ coli_status check_layer(const coli_moe_layer* L, int T)
         return fail(COLI_ERR_UNSUPPORTED, "hidden=%d / ffn=%d above %d", L->hidden, L->ffn, kMaxStageK);
     if (!std::isfinite(L->routed_scale)) return fail(COLI_ERR_INVALID_ARG, "routed_scale is not finite");
     if (!(L->top_p >= 0.f) || !std::isfinite(L->top_p)) return fail(COLI_ERR_INVALID_ARG, "top_p is negative or not finite");
+    if (L->act_int8 != 0 && L->act_int8 != 1) return fail(COLI_ERR_INVALID_ARG, "act_int8=%d (0 or 1)", L->act_int8);
     const void* ptrs[] = {L->w_router, L->sel_bias, L->gate_q, L->up_q, L->down_q, L->gate_s, L->up_s, L->down_s};
     const char* names[] = {"w_router", "sel_bias", "gate_q", "up_q", "down_q", "gate_s", "up_s", "down_s"};
     for (int i = 0; i < 8; ++i) {
@@ -258,6 +259,8 @@ coli_status check_layer(const coli_moe_layer* L, int T)
 }
 
 // Argument checks of a layer call other than its workspace (host only).
+int choose_path(const coli_moe_layer* L, int T);
+
 coli_status check_call(const coli_moe_layer* L, const void* x, coli_dtype xt, int T, const void* out, coli_dtype ot,
                        const int32_t* topk_idx_out, const float* topk_w_out)
 {
@@ -266,6 +269,12 @@ coli_status check_call(const coli_moe_layer* L, const void* x, coli_dtype xt, in
     if (xt != COLI_F32 && xt != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown activation dtype %d", (int)xt);
     if (ot != COLI_F32 && ot != COLI_BF16) return fail(COLI_ERR_INVALID_ARG, "unknown output dtype %d", (int)ot);
     if (T == 0) return COLI_OK;
+    if (L->act_int8) {
+        const int p = choose_path(L, T);
+        if (p != COLI_PATH_SINGLE && p != COLI_PATH_DECODE)
+            return fail(COLI_ERR_UNSUPPORTED, "act_int8: the integer-activation variant runs in the fused decode kernel "
+                                              "(batches of up to %d tokens)", kDecodeMaxT);
+    }
     if (!x || !out) return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned(x, 16) || !aligned(out, 16)) return fail(COLI_ERR_INVALID_ARG, "x / out not 16-byte aligned");
     if ((topk_idx_out && !aligned(topk_idx_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
@@ -555,7 +564,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
             return cuda_fail(e, "event record");
         LayerArgs la{L->w_router, L->sel_bias, L->gate_q, L->gate_s, L->up_q, L->up_s, L->down_q, L->down_s,
                      H, F, E, k, T, L->routed_scale, x, out, w.logits, fused_router ? 0 : 1, idx, wt, w.h,
-                     w.partial, w.ctl + 3, wait_limit(kBarrierNs), L->top_p, g_stamps.load()};
+                     w.partial, w.ctl + 3, wait_limit(kBarrierNs), L->top_p, g_stamps.load(), L->act_int8};
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(dev->sms);
         cfg.blockDim = dim3(layer_threads(pl.MT));

@@ -245,6 +245,10 @@ static __device__ __noinline__ void stage_rows(const void* __restrict__ src, int
 // integer products leave the float pipes free and take far fewer issue slots
 // than decoding nibbles to floats.
 //
+// The integer-activation variant (int8 activations) uses the first plane pair
+// only: d0 = round(x * 127 / m), scale m / 127 (the pages' integer dot-product
+// kernel, "Colibri 完全ガイド", section コア技術のハイライト).
+//
 // Shared-memory layout of one staged vector: chunk c = l + 32 i, plane
 // p = 2 * digit + (0: lo, 1: hi), as uint4 at ((i * 6 + p) * 32 + l); word w
 // of the uint4 covers k = 8 w .. 8 w + 7 of the chunk, byte b of a lo (hi)
@@ -291,7 +295,7 @@ __device__ __forceinline__ uint32_t pack_lo_bytes(uint32_t a, uint32_t b, uint32
 // one copy of the code serves every call site.
 static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ src, int bf16, int K, int n, int row0,
                                                       const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
-                                                      int nthr)
+                                                      int nthr, int i8)
 {
     const int nch = K / kChunkK;
     const int vunits = digit_vec_units(K);
@@ -328,6 +332,32 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
 #pragma unroll
         for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(x[j]));
         const bool finite = m <= 3.402823466e38f;  // false for inf and NaN
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
+        if (i8) {
+            // integer-activation variant: one plane of symmetric int8 codes, scale max / 127 (a block
+            // whose 127 / max overflows is zero)
+            const float inv = finite && m > 0.f ? 127.0f / m : 0.f;
+            const bool live8 = inv <= 3.402823466e38f && inv > 0.f;
+            int csum8 = 0;
+            uint32_t X8[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int v = live8 ? (int)fminf(fmaxf(rintf(x[j] * inv), -127.f), 127.f) : 0;
+                X8[j] = (uint32_t)v;
+                csum8 += v;
+            }
+            uint32_t lo8[4], hi8[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                lo8[w] = pack_lo_bytes(X8[8 * w], X8[8 * w + 2], X8[8 * w + 4], X8[8 * w + 6]);
+                hi8[w] = pack_lo_bytes(X8[8 * w + 1], X8[8 * w + 3], X8[8 * w + 5], X8[8 * w + 7]);
+            }
+            base[0] = make_uint4(lo8[0], lo8[1], lo8[2], lo8[3]);
+            base[32] = make_uint4(hi8[0], hi8[1], hi8[2], hi8[3]);
+            const float scale8 = !finite ? __int_as_float(0x7FC00000) : live8 ? m / 127.0f : 0.f;
+            xc[(size_t)t * nch + c] = make_float2(scale8, __int_as_float(8 * csum8));
+            continue;
+        }
         const int ex = (int)(__float_as_uint(m) >> 23);
         // chunks whose largest magnitude is below 2^-100 contribute nothing (their products are far below any
         // fp32 rounding of the result); e = ex - 126 gives m < 2^e
@@ -344,7 +374,6 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
             X[j] = (uint32_t)vc;
             csum += vc;
         }
-        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
         uint32_t lo[4], hi[4];
         // plane d2: bits 0-6; d1: bits 7-13; d0: bits 14-21 (signed)
 #pragma unroll

@@ -131,7 +131,7 @@ struct VecSet {
 template <int MT>
 __device__ __forceinline__ void chunk_pair_digit_vectors(const uint4& w0, const uint4& w1, const uint4* xd,
                                                          const float2* cc, const VecSet<MT>& v, int vstride, int nch,
-                                                         float s0, float s1, float (&tot)[2][MT])
+                                                         int nd, float s0, float s1, float (&tot)[2][MT])
 {
     uint32_t al[4], ah[4], bl[4], bh[4];
 #pragma unroll
@@ -150,21 +150,28 @@ __device__ __forceinline__ void chunk_pair_digit_vectors(const uint4& w0, const 
             int a0[3] = {0, 0, 0}, a1[3] = {0, 0, 0};
 #pragma unroll
             for (int d = 0; d < 3; ++d) {
-                const uint4 xl = x[(2 * d) * 32], xh = x[(2 * d + 1) * 32];
+                if (d < nd) {
+                    const uint4 xl = x[(2 * d) * 32], xh = x[(2 * d + 1) * 32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t l = q == 0 ? xl.x : q == 1 ? xl.y : q == 2 ? xl.z : xl.w;
-                    const uint32_t h = q == 0 ? xh.x : q == 1 ? xh.y : q == 2 ? xh.z : xh.w;
-                    a0[d] = dp4a_us(al[q], l, a0[d]);
-                    a0[d] = dp4a_us(ah[q], h, a0[d]);
-                    a1[d] = dp4a_us(bl[q], l, a1[d]);
-                    a1[d] = dp4a_us(bh[q], h, a1[d]);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t l = q == 0 ? xl.x : q == 1 ? xl.y : q == 2 ? xl.z : xl.w;
+                        const uint32_t h = q == 0 ? xh.x : q == 1 ? xh.y : q == 2 ? xh.z : xh.w;
+                        a0[d] = dp4a_us(al[q], l, a0[d]);
+                        a0[d] = dp4a_us(ah[q], h, a0[d]);
+                        a1[d] = dp4a_us(bl[q], l, a1[d]);
+                        a1[d] = dp4a_us(bh[q], h, a1[d]);
+                    }
                 }
             }
             const float2 c = cc[v.vi[t] * nch];
             const uint32_t corr = (uint32_t)__float_as_int(c.y);
-            const uint32_t D0 = ((uint32_t)a0[0] * 128u + (uint32_t)a0[1]) * 128u + (uint32_t)a0[2] - corr;
-            const uint32_t D1 = ((uint32_t)a1[0] * 128u + (uint32_t)a1[1]) * 128u + (uint32_t)a1[2] - corr;
+            uint32_t D0 = (uint32_t)a0[0], D1 = (uint32_t)a1[0];
+            if (nd == 3) {  // X = 16384 d0 + 128 d1 + d2; one plane: X = d0
+                D0 = (D0 * 128u + (uint32_t)a0[1]) * 128u + (uint32_t)a0[2];
+                D1 = (D1 * 128u + (uint32_t)a1[1]) * 128u + (uint32_t)a1[2];
+            }
+            D0 -= corr;
+            D1 -= corr;
             tot[0][t] = fmaf(s0 * c.x, (float)(int)D0, tot[0][t]);
             tot[1][t] = fmaf(s1 * c.x, (float)(int)D1, tot[1][t]);
         }
@@ -234,7 +241,7 @@ __device__ __forceinline__ float lds32(uint32_t smem)
 
 template <int MT, int R, typename RowsOf, typename VecsOf, typename Finish, typename Hook = NoHook>
 __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per_lane, int nch, const float4* xs,
-                                                 const void* corr, unsigned char* ring, RowsOf rows_of,
+                                                 const void* corr, int nd, unsigned char* ring, RowsOf rows_of,
                                                  VecsOf vecs_of, Finish finish, Hook hook = Hook())
 {
     if (nj <= 0) {
@@ -305,7 +312,7 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
         if (whole || lane + 32 * cci < nch) {
             const uint4 w0 = lds128(csl), w1 = lds128(csl + 512);
             const float s0 = lds32(csl + sc_off), s1 = lds32(csl + sc_off + 128);
-            chunk_pair_digit_vectors<MT>(w0, w1, xrow, crow, v, vstride, nch, s0, s1, tot);
+            chunk_pair_digit_vectors<MT>(w0, w1, xrow, crow, v, vstride, nch, nd, s0, s1, tot);
         }
         csl += kSlotBytes;
         if (csl == ring_end) csl = ring_lane;
@@ -350,6 +357,7 @@ struct LayerArgs {
     unsigned long long wait_ns;  // limit of each grid-barrier wait
     float top_p;            // adaptive expert top-p (0: plain top-k)
     unsigned long long* stamps;  // optional [gridDim.x, kStamps] globaltimer stamps per CTA (test hook)
+    int act_i8;             // integer-activation variant: int8 activations per 32 (one digit plane)
 };
 
 constexpr int kStamps = 16;
@@ -836,6 +844,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
+    const int nd = a.act_i8 ? 1 : 3;  // digit planes per staged vector (int8 variant: one)
     // staged vectors as digit planes (16-byte units per vector)
     const int xvs = digit_vec_units(H);
     const int hvs = digit_vec_units(F);
@@ -862,7 +871,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     auto stage_vecs = [&](const void* src, int bf16, int K, int n, int row0, const int* tbl, int tdiv, float4* dst,
                           unsigned char* dcorr, int tid, int nthr) {
         stage_rows_digits(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
-                          reinterpret_cast<float2*>(dcorr), tid, nthr);
+                          reinterpret_cast<float2*>(dcorr), tid, nthr, a.act_i8);
     };
     auto stage_x = [&](int n, int row0, const int* tbl = nullptr, int tdiv = 1) {
         stage_vecs(a.x, kBf16 ? 1 : 0, H, n, row0, tbl, tdiv, xs, xcorr, (int)threadIdx.x, kLayerThreads);
@@ -951,7 +960,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
+            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of,
                                        fin, hook);
             ran = true;
         }
@@ -1060,7 +1069,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             };
             const int first = warp;
             const int nj = first < npr ? (npr - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of,
+            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of,
                                        fin, route_hook);
         }
         stamp(a, 14);
@@ -1094,7 +1103,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         };
         const int first = lo + warp;
         const int nj = first < hi ? (hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-        stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of, fin);
+        stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of, fin);
     } else {
         const bool scored_here = all_x;  // the kernel scored the tokens (pieces summed into shared memory)
         if (scored_here) sum_pieces();
@@ -1216,7 +1225,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin);
+            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin);
         }
 
         // routed gate/up: one run over all routed groups when every token is staged,
@@ -1264,7 +1273,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of, fin);
+            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of, fin);
         }
     }
     stamp(a, 5);
@@ -1312,7 +1321,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int total = npr * n_kept;
         const int first = warp;
         const int nj = first < total ? (total - first + kLayerWarps - 1) / kLayerWarps : 0;
-        stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin,
+        stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin,
                                    hook);
         __syncthreads();
         stamp(a, 8);
@@ -1377,7 +1386,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin);
+            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin);
         }
         grid_barrier(bar, deadline, a.err);
 

@@ -101,10 +101,20 @@ def test_status_word_offset(coli):
     (dict(top_k=33), 1), (dict(n_experts=4, top_k=8), 1), (dict(n_experts=2000), 1),
     (dict(group=128), 2), (dict(hidden=32768), 2), (dict(w_router=0), 1), (dict(gate_q=(1 << 20) + 8), 1),
     (dict(routed_scale=float("inf")), 1), (dict(top_p=-0.5), 1), (dict(top_p=float("nan")), 1),
+    (dict(act_int8=2), 1), (dict(act_int8=-1), 1),
 ])
 def test_forward_rejects_bad_layers(coli, over, status):
     assert _fwd(coli, _layer(coli, **over)) == status
     assert coli.last_error() != ""
+
+
+def test_int8_activations_only_in_the_decode_kernel(coli):
+    """The integer-activation variant runs in the fused decode kernel; a batch
+    that goes to another chain is refused before anything is launched."""
+    s = _layer(coli, act_int8=1)
+    assert _fwd(coli, s, T=65) == 2
+    assert "act_int8" in coli.last_error()
+    assert _fwd(coli, s, T=4096) == 2
 
 
 def test_forward_rejects_bad_calls(coli):

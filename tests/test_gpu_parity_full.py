@@ -113,3 +113,33 @@ def test_full_size_layer_matches_oracle(full, cfg):
     _, _, rout = oracle.moe_layer(x[tokens], c.H, c.F, c.E, c.k, c.routed_scale, w_router, sel_bias, experts)
     tol = S.TOL_PREFILL if T > 64 else S.TOL_DECODE
     S.check_output(out[tokens], rout, tol, f"{c.name} ({len(tokens)} of {T} tokens)")
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_full_size_int8_activations_match_oracle(full, cfg):
+    """The integer-activation variant (layer.act_int8) at the full shape, every
+    token: routing bit-exact, output against the oracle's int8-activation layer
+    within the decode tolerance (the quantisation is reproduced exactly; an h
+    value within fp32 rounding of a code boundary may take the other code,
+    which moves the output by about 0.03 / sqrt(F) of its norm)."""
+    coli, torch, bufs, host_expert = full
+    c = inputs.CONFIGS[cfg]
+    w_router, sel_bias = inputs.router_params(c, SEED, LAYER)
+    x, _ = S.x_without_ties(c, SEED, 1, LAYER, w_router, sel_bias)
+    L = coli.Layer(c.H, c.F, c.E, c.k, c.routed_scale, torch.from_numpy(w_router).cuda(),
+                   torch.from_numpy(sel_bias).cuda(), bufs["gate_q"], bufs["gate_s"], bufs["up_q"],
+                   bufs["up_s"], bufs["down_q"], bufs["down_s"], act_int8=True)
+    T = c.T
+    out = torch.empty((T, c.H), dtype=torch.bfloat16 if c.out_dtype == "bf16" else torch.float32,
+                      device="cuda")
+    ws = torch.empty(coli.moe_workspace_size(L, T), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((T, c.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, c.k), dtype=torch.float32, device="cuda")
+    coli.moe_forward(L, S.to_device_x(x, torch), out, ws, idx, w)
+    torch.cuda.synchronize()
+    ridx, rw = oracle.route(x, w_router, sel_bias, c.k, c.routed_scale)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    need = set(ridx.ravel().tolist()) | {c.E}
+    experts = {e: host_expert(e) for e in need}
+    _, _, rout = oracle.moe_layer_i8(x, c.H, c.F, c.E, c.k, c.routed_scale, w_router, sel_bias, experts)
+    S.check_output(S.output_to_f64(out, torch), rout, S.TOL_DECODE, f"{c.name} int8 activations")
