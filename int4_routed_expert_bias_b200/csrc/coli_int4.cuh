@@ -295,7 +295,7 @@ __device__ __forceinline__ uint32_t pack_lo_bytes(uint32_t a, uint32_t b, uint32
 // one copy of the code serves every call site.
 static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ src, int bf16, int K, int n, int row0,
                                                       const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
-                                                      int nthr, int i8)
+                                                      int nthr)
 {
     const int nch = K / kChunkK;
     const int vunits = digit_vec_units(K);
@@ -332,32 +332,6 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
 #pragma unroll
         for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(x[j]));
         const bool finite = m <= 3.402823466e38f;  // false for inf and NaN
-        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
-        if (i8) {
-            // integer-activation variant: one plane of symmetric int8 codes, scale max / 127 (a block
-            // whose 127 / max overflows is zero)
-            const float inv = finite && m > 0.f ? 127.0f / m : 0.f;
-            const bool live8 = inv <= 3.402823466e38f && inv > 0.f;
-            int csum8 = 0;
-            uint32_t X8[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int v = live8 ? (int)fminf(fmaxf(rintf(x[j] * inv), -127.f), 127.f) : 0;
-                X8[j] = (uint32_t)v;
-                csum8 += v;
-            }
-            uint32_t lo8[4], hi8[4];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                lo8[w] = pack_lo_bytes(X8[8 * w], X8[8 * w + 2], X8[8 * w + 4], X8[8 * w + 6]);
-                hi8[w] = pack_lo_bytes(X8[8 * w + 1], X8[8 * w + 3], X8[8 * w + 5], X8[8 * w + 7]);
-            }
-            base[0] = make_uint4(lo8[0], lo8[1], lo8[2], lo8[3]);
-            base[32] = make_uint4(hi8[0], hi8[1], hi8[2], hi8[3]);
-            const float scale8 = !finite ? __int_as_float(0x7FC00000) : live8 ? m / 127.0f : 0.f;
-            xc[(size_t)t * nch + c] = make_float2(scale8, __int_as_float(8 * csum8));
-            continue;
-        }
         const int ex = (int)(__float_as_uint(m) >> 23);
         // chunks whose largest magnitude is below 2^-100 contribute nothing (their products are far below any
         // fp32 rounding of the result); e = ex - 126 gives m < 2^e
@@ -374,6 +348,7 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
             X[j] = (uint32_t)vc;
             csum += vc;
         }
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
         uint32_t lo[4], hi[4];
         // plane d2: bits 0-6; d1: bits 7-13; d0: bits 14-21 (signed)
 #pragma unroll
@@ -400,6 +375,74 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
         base[1 * 32] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         const float scale = !finite ? __int_as_float(0x7FC00000) : live ? __uint_as_float((uint32_t)(106 + e) << 23)
                                                                           : 0.f;
+        xc[(size_t)t * nch + c] = make_float2(scale, __int_as_float(8 * csum));
+    }
+}
+
+// The integer-activation variant's staging: one plane pair of symmetric int8
+// codes per chunk, code = rint(x * (127 / m)) with m = max |x| of the chunk,
+// scale m / 127 (a chunk whose 127 / m overflows fp32 is zero; one holding inf
+// or NaN gets scale NaN).  Same layout as stage_rows_digits (first plane pair,
+// a float2 (scale, 8 * sum of codes) per chunk).
+static __device__ __noinline__ void stage_rows_int8(const void* __restrict__ src, int bf16, int K, int n, int row0,
+                                                    const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
+                                                    int nthr)
+{
+    const int nch = K / kChunkK;
+    const int vunits = digit_vec_units(K);
+    const size_t row_bytes = (size_t)K * (bf16 ? 2 : 4);
+    for (int idx = tid; idx < n * nch; idx += nthr) {
+        const int t = idx / nch, c = idx - t * nch;
+        const int row = tbl ? tbl[t] / tdiv : row0 + t;
+        const char* rp = static_cast<const char*>(src) + (size_t)row * row_bytes;
+        float x[32];
+        if (bf16) {
+            const uint4* p4 = reinterpret_cast<const uint4*>(rp + (size_t)c * kChunkK * 2);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v = p4[j];
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    x[8 * j + 2 * h] = bf16_bits_to_float(u[h] & 0xFFFFu);
+                    x[8 * j + 2 * h + 1] = bf16_bits_to_float(u[h] >> 16);
+                }
+            }
+        } else {
+            const float4* p4 = reinterpret_cast<const float4*>(rp + (size_t)c * kChunkK * 4);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 v = p4[j];
+                x[4 * j] = v.x;
+                x[4 * j + 1] = v.y;
+                x[4 * j + 2] = v.z;
+                x[4 * j + 3] = v.w;
+            }
+        }
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(x[j]));
+        const bool finite = m <= 3.402823466e38f;  // false for inf and NaN
+        const float inv = finite && m > 0.f ? 127.0f / m : 0.f;
+        const bool live = inv > 0.f && inv <= 3.402823466e38f;
+        uint32_t X[32];
+        int csum = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int v = live ? (int)fminf(fmaxf(rintf(x[j] * inv), -127.f), 127.f) : 0;
+            X[j] = (uint32_t)v;
+            csum += v;
+        }
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            lo[w] = pack_lo_bytes(X[8 * w], X[8 * w + 2], X[8 * w + 4], X[8 * w + 6]);
+            hi[w] = pack_lo_bytes(X[8 * w + 1], X[8 * w + 3], X[8 * w + 5], X[8 * w + 7]);
+        }
+        base[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        base[32] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        const float scale = !finite ? __int_as_float(0x7FC00000) : live ? m / 127.0f : 0.f;
         xc[(size_t)t * nch + c] = make_float2(scale, __int_as_float(8 * csum));
     }
 }

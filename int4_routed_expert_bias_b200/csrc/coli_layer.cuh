@@ -870,8 +870,12 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     // activations / SwiGLU outputs into shared memory: vector t = row row0 + t (or tbl[t] / tdiv)
     auto stage_vecs = [&](const void* src, int bf16, int K, int n, int row0, const int* tbl, int tdiv, float4* dst,
                           unsigned char* dcorr, int tid, int nthr) {
-        stage_rows_digits(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
-                          reinterpret_cast<float2*>(dcorr), tid, nthr, a.act_i8);
+        if (a.act_i8)
+            stage_rows_int8(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
+                            reinterpret_cast<float2*>(dcorr), tid, nthr);
+        else
+            stage_rows_digits(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
+                              reinterpret_cast<float2*>(dcorr), tid, nthr);
     };
     auto stage_x = [&](int n, int row0, const int* tbl = nullptr, int tdiv = 1) {
         stage_vecs(a.x, kBf16 ? 1 : 0, H, n, row0, tbl, tdiv, xs, xcorr, (int)threadIdx.x, kLayerThreads);
