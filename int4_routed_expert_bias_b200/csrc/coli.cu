@@ -98,20 +98,23 @@ cudaError_t allow_smem(Kern k, int bytes)
 }
 
 // The fused decode-layer kernel, one instantiation per (tokens per group,
-// activation dtype, output dtype, one-token output-row mode).
+// activation dtype, output dtype, one-token output-row mode, int8 activations).
 using LayerKernel = void (*)(const LayerArgs, const LayerSmem);
-LayerKernel layer_kernel(int MT, bool bf16, bool out_bf16, bool out_rows)
+template <int MT, bool kRows, bool kI8>
+LayerKernel layer_kernel_dtypes(bool bf16, bool out_bf16)
 {
-    if (MT == 4) {
-        if (bf16) return out_bf16 ? moe_layer_kernel<4, true, true, false> : moe_layer_kernel<4, true, false, false>;
-        return out_bf16 ? moe_layer_kernel<4, false, true, false> : moe_layer_kernel<4, false, false, false>;
-    }
-    if (out_rows) {
-        if (bf16) return out_bf16 ? moe_layer_kernel<1, true, true, true> : moe_layer_kernel<1, true, false, true>;
-        return out_bf16 ? moe_layer_kernel<1, false, true, true> : moe_layer_kernel<1, false, false, true>;
-    }
-    if (bf16) return out_bf16 ? moe_layer_kernel<1, true, true, false> : moe_layer_kernel<1, true, false, false>;
-    return out_bf16 ? moe_layer_kernel<1, false, true, false> : moe_layer_kernel<1, false, false, false>;
+    if (bf16)
+        return out_bf16 ? moe_layer_kernel<MT, true, true, kRows, kI8> : moe_layer_kernel<MT, true, false, kRows, kI8>;
+    return out_bf16 ? moe_layer_kernel<MT, false, true, kRows, kI8> : moe_layer_kernel<MT, false, false, kRows, kI8>;
+}
+
+LayerKernel layer_kernel(int MT, bool bf16, bool out_bf16, bool out_rows, bool i8)
+{
+    if (MT == 4)
+        return i8 ? layer_kernel_dtypes<4, false, true>(bf16, out_bf16) : layer_kernel_dtypes<4, false, false>(bf16, out_bf16);
+    if (out_rows)
+        return i8 ? layer_kernel_dtypes<1, true, true>(bf16, out_bf16) : layer_kernel_dtypes<1, true, false>(bf16, out_bf16);
+    return i8 ? layer_kernel_dtypes<1, false, true>(bf16, out_bf16) : layer_kernel_dtypes<1, false, false>(bf16, out_bf16);
 }
 
 cudaError_t allow_layer_kernels(int bytes)
@@ -119,9 +122,9 @@ cudaError_t allow_layer_kernels(int bytes)
     const int mts[2] = {1, 4};
     for (int mt : mts)
         for (int rows = 0; rows < 2; ++rows)
-            for (int b = 0; b < 4; ++b) {
+            for (int b = 0; b < 8; ++b) {
                 if (mt == 4 && rows) continue;
-                const cudaError_t e = cudaFuncSetAttribute(layer_kernel(mt, b & 1, b & 2, rows),
+                const cudaError_t e = cudaFuncSetAttribute(layer_kernel(mt, b & 1, b & 2, rows, b & 4),
                                                            cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
                 if (e != cudaSuccess) return e;
             }
@@ -548,7 +551,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     if (path == COLI_PATH_SINGLE || path == COLI_PATH_DECODE) {
         const LayerPlan pl = layer_plan(T, H, F, E, k);
         if (dev->sms < kMinLayerSms) return fail(COLI_ERR_UNSUPPORTED, "%d SMs: the decode kernel needs %d", dev->sms, kMinLayerSms);
-        const LayerKernel kern = layer_kernel(pl.MT, bf16, ot == COLI_BF16, pl.out_rows);
+        const LayerKernel kern = layer_kernel(pl.MT, bf16, ot == COLI_BF16, pl.out_rows, L->act_int8 != 0);
         int occ = 0;
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, layer_threads(pl.MT), pl.ls.bytes)) != cudaSuccess)
             return cuda_fail(e, "occupancy query");
@@ -564,7 +567,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
             return cuda_fail(e, "event record");
         LayerArgs la{L->w_router, L->sel_bias, L->gate_q, L->gate_s, L->up_q, L->up_s, L->down_q, L->down_s,
                      H, F, E, k, T, L->routed_scale, x, out, w.logits, fused_router ? 0 : 1, idx, wt, w.h,
-                     w.partial, w.ctl + 3, wait_limit(kBarrierNs), L->top_p, g_stamps.load(), L->act_int8};
+                     w.partial, w.ctl + 3, wait_limit(kBarrierNs), L->top_p, g_stamps.load()};
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(dev->sms);
         cfg.blockDim = dim3(layer_threads(pl.MT));

@@ -79,7 +79,7 @@ __device__ __forceinline__ GridBar grid_bar_open(unsigned int* word)
     if (threadIdx.x == 0) {
         unsigned int cur;
         asm volatile("ld.relaxed.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(word) : "memory");
-        b.phase = cur & 0x80000000u;
+        b.phase = cur;  // only bit 31 is compared; the value is first needed at the first barrier
     }
     return b;
 }
@@ -357,7 +357,6 @@ struct LayerArgs {
     unsigned long long wait_ns;  // limit of each grid-barrier wait
     float top_p;            // adaptive expert top-p (0: plain top-k)
     unsigned long long* stamps;  // optional [gridDim.x, kStamps] globaltimer stamps per CTA (test hook)
-    int act_i8;             // integer-activation variant: int8 activations per 32 (one digit plane)
 };
 
 constexpr int kStamps = 16;
@@ -829,8 +828,9 @@ __device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, i
 __device__ __forceinline__ int pair_cost(int K, int m) { return max(1, (K + K / 8) / 256) * (3 + m); }
 
 // The layer, T <= 64 tokens.  MT = tokens per group (vectors per item);
-// kOutRows: one token, down and combine by output rows.
-template <int MT, bool kBf16, bool kOutBf16, bool kOutRows>
+// kOutRows: one token, down and combine by output rows; kI8: the
+// integer-activation variant (int8 activations, one digit plane).
+template <int MT, bool kBf16, bool kOutBf16, bool kOutRows, bool kI8>
 __global__ void __launch_bounds__(layer_threads(MT), 1)
 moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 {
@@ -844,7 +844,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
-    const int nd = a.act_i8 ? 1 : 3;  // digit planes per staged vector (int8 variant: one)
+    constexpr int nd = kI8 ? 1 : 3;  // digit planes per staged vector (int8 variant: one)
     // staged vectors as digit planes (16-byte units per vector)
     const int xvs = digit_vec_units(H);
     const int hvs = digit_vec_units(F);
@@ -870,7 +870,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     // activations / SwiGLU outputs into shared memory: vector t = row row0 + t (or tbl[t] / tdiv)
     auto stage_vecs = [&](const void* src, int bf16, int K, int n, int row0, const int* tbl, int tdiv, float4* dst,
                           unsigned char* dcorr, int tid, int nthr) {
-        if (a.act_i8)
+        if constexpr (kI8)
             stage_rows_int8(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
                             reinterpret_cast<float2*>(dcorr), tid, nthr);
         else
@@ -917,14 +917,25 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             stamp(a, 1);
         };
         const int nseg = n_sg;
-        for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
-            u.seg_i[s] = F;
-            u.seg_cost[s] = pair_cost(H, min(MT, T - s * MT));
-        }
-        __syncthreads();
-        const SegTable st = seg_prepare(u, nseg);
+        SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
         int lo, hi;
-        seg_cta_range(st, lo, hi);
+        if (nseg == 1) {  // one token group: an even split of the F row pairs
+            if (threadIdx.x == 0) {
+                u.seg_i[0] = 0;
+                u.seg_i[1] = F;
+            }
+            __syncthreads();
+            lo = (int)((long long)F * blockIdx.x / gridDim.x);
+            hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
+        } else {
+            for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
+                u.seg_i[s] = F;
+                u.seg_cost[s] = pair_cost(H, min(MT, T - s * MT));
+            }
+            __syncthreads();
+            st = seg_prepare(u, nseg);
+            seg_cta_range(st, lo, hi);
+        }
         stamp(a, 10);
         bool ran = false;
         for (int s = 0; s < nseg; ++s) {
