@@ -147,13 +147,13 @@ COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
  * kept experts, dropped slots are reported as index -1 with weight 0 and cost
  * no expert reads.  The rule is this library's reading: the page names the
  * knob and its effect only.  The router is fp32.  Batches of up to 64 tokens
- * compute the experts in fp32 (bf16 x is widened exactly); larger batches run
- * them on the tensor cores with bf16 operands (weights q * scale, activations
- * and the SwiGLU output rounded to bf16) and fp32 accumulation.  In the
- * 1-64-token kernel the activations enter the expert products as 21-bit fixed
- * point per block of 32 values (power-of-two block scale; each value within
- * 2^-21 of its block's largest magnitude) with exact integer products, an
- * error of the same order as fp32 arithmetic.
+ * compute the experts with fp32 accumulation; the activations (and the SwiGLU
+ * output h) enter the expert products as 21-bit fixed point per block of 32
+ * values (power-of-two block scale; each value within 2^-21 of its block's
+ * largest magnitude), multiplied exactly in integers: an error of the order of
+ * fp32 arithmetic.  Larger batches run the experts on the tensor cores with
+ * bf16 operands (weights q * scale, activations and the SwiGLU output rounded
+ * to bf16) and fp32 accumulation.
  * Integer-activation variant (layer->act_int8 = 1; "Colibri 完全ガイド", section
  * コア技術のハイライト, row 整数ドット積カーネル, int8 activations times packed
  * int4 weights): x before gate/up and h before down are quantised to
