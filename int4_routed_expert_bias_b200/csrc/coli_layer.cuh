@@ -781,34 +781,42 @@ __device__ __forceinline__ unsigned int* launch_barrier_word()
     return ws ? &ws->barrier : nullptr;
 }
 
-// Partial router scores of one piece: chunks c = lane + 32 p of router row e
-// (32 fp32 weights each) against the nt tokens' activations, read in fp32 from
-// global memory (L2); the warp's sums go to logit_part[p][t][e].
-template <int NT, bool kBf16>
+// Partial router scores of one piece: chunks c = lane + 32 (PC p + q), q < PC,
+// of router row e (32 fp32 weights each) against the nt tokens' activations,
+// read in fp32 from global memory (L2); the warp's sums go to
+// logit_part[p][t][e].  All the piece's weight loads are issued together.
+template <int NT, bool kBf16, int PC>
 __device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, int nt, const StageGeom& g)
 {
     const int lane = threadIdx.x & 31;
-    const int c = lane + 32 * p;
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-    if (c < g.nch) {
+    const uint64_t pol = l2_evict_first();
+    float4 wv[PC][8];
+#pragma unroll
+    for (int q = 0; q < PC; ++q) {
+        const int c = lane + 32 * (PC * p + q);
         const float4* wrow = reinterpret_cast<const float4*>(a.w_router + (size_t)e * a.H) + (size_t)c * 8;
-        const uint64_t pol = l2_evict_first();
-        float4 wv[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) wv[j] = ldg_stream4(wrow + j, pol);
+        for (int j = 0; j < 8; ++j) wv[q][j] = c < g.nch ? ldg_stream4(wrow + j, pol) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            if (t < nt) {
-                const char* xr = static_cast<const char*>(a.x) + (size_t)t * a.H * (kBf16 ? 2 : 4);
+    for (int q = 0; q < PC; ++q) {
+        const int c = lane + 32 * (PC * p + q);
+        if (c < g.nch) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 xv = load_act4<kBf16>(xr, c * kChunkK + 4 * j);
-                    acc[t] = fmaf(wv[j].x, xv.x, acc[t]);
-                    acc[t] = fmaf(wv[j].y, xv.y, acc[t]);
-                    acc[t] = fmaf(wv[j].z, xv.z, acc[t]);
-                    acc[t] = fmaf(wv[j].w, xv.w, acc[t]);
+            for (int t = 0; t < NT; ++t) {
+                if (t < nt) {
+                    const char* xr = static_cast<const char*>(a.x) + (size_t)t * a.H * (kBf16 ? 2 : 4);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 xv = load_act4<kBf16>(xr, c * kChunkK + 4 * j);
+                        acc[t] = fmaf(wv[q][j].x, xv.x, acc[t]);
+                        acc[t] = fmaf(wv[q][j].y, xv.y, acc[t]);
+                        acc[t] = fmaf(wv[q][j].z, xv.z, acc[t]);
+                        acc[t] = fmaf(wv[q][j].w, xv.w, acc[t]);
+                    }
                 }
             }
         }
@@ -845,6 +853,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
     constexpr int nd = kI8 ? 1 : 3;  // digit planes per staged vector (int8 variant: one)
+    constexpr int kPieceChunks = MT == 1 ? 2 : 1;  // router chunks per lane per piece
     // staged vectors as digit planes (16-byte units per vector)
     const int xvs = digit_vec_units(H);
     const int hvs = digit_vec_units(F);
@@ -905,21 +914,28 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         // warps one each, so every block has about the same number.  The shared expert's gate/up
         // rows are cut into equal-cost ranges.  The first gate/up loads are issued before the
         // activations are staged and before the warp's router piece is computed (engine hook).
-        const int nrp = a.n_pieces == 0 ? gH.per_lane : 0;  // router pieces per row (computed here)
+        const int nrp = a.n_pieces == 0 ? (gH.per_lane + kPieceChunks - 1) / kPieceChunks : 0;  // pieces per row
+        // The router pieces read the activations from global memory and are needed only after the
+        // grid barrier, so a warp takes its pieces after its gate/up items (their loads overlap the
+        // other warps' streams); the warps are dealt the pieces from the last warp down, since the
+        // first warps hold the gate/up items.
         auto router_pieces = [&]() {
             const int total = E * nrp;
-            for (int i = blockIdx.x + gridDim.x * warp; i < total; i += gridDim.x * kLayerWarps)
-                router_piece<MT, kBf16>(a, i / nrp, i % nrp, T, gH);
+            for (int i = blockIdx.x + gridDim.x * (kLayerWarps - 1 - warp); i < total; i += gridDim.x * kLayerWarps)
+                router_piece<MT, kBf16, kPieceChunks>(a, i / nrp, i % nrp, T, gH);
         };
         auto stage_all = [&]() {
             stage_x(T, 0);
             __syncthreads();
             stamp(a, 1);
         };
-        const int nseg = n_sg;
+        // one token: the activations and the router only; the shared expert's rows stream in phase B
+        // (their first loads in flight while the token is routed) and C
+        const int nseg = kOutRows ? 0 : n_sg;
         SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
-        int lo, hi;
-        if (nseg == 1) {  // one token group: an even split of the F row pairs
+        int lo = 0, hi = 0;
+        if (kOutRows) {
+        } else if (nseg == 1) {  // one token group: an even split of the F row pairs
             if (threadIdx.x == 0) {
                 u.seg_i[0] = 0;
                 u.seg_i[1] = F;
@@ -963,10 +979,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             };
             auto hook = [&]() {
                 if (all_x) {
-                    if (!ran) {
-                        stage_all();
-                        router_pieces();
-                    }
+                    if (!ran) stage_all();
                 } else {  // this group's tokens (the router ran before the launch)
                     __syncthreads();
                     stage_x(m, t0);
@@ -979,9 +992,24 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                                        fin, hook);
             ran = true;
         }
-        if (!ran && all_x) {  // no gate/up rows in this block: activations and router pieces only
-            stage_all();
-            router_pieces();
+        if constexpr (kOutRows) {
+            // one token, nothing streams in this phase: the router pieces (their weight loads the longest
+            // latency here) run on the last rw warps beside the staging of x on the others
+            const int per_cta = (E * nrp + (int)gridDim.x - 1) / (int)gridDim.x;
+            const int rw = max(1, min(kLayerWarps - 4, per_cta));
+            const int xw = kLayerWarps - rw;
+            if (warp < xw) {
+                stage_vecs(a.x, kBf16 ? 1 : 0, H, 1, 0, nullptr, 1, xs, xcorr, (int)threadIdx.x, xw * 32);
+            } else {
+                const int total = E * nrp;
+                for (int i = blockIdx.x + gridDim.x * (warp - xw); i < total; i += gridDim.x * rw)
+                    router_piece<MT, kBf16, kPieceChunks>(a, i / nrp, i % nrp, T, gH);
+            }
+            __syncthreads();
+            stamp(a, 1);
+        } else {
+            if (!ran && all_x) stage_all();  // no gate/up rows in this block: the activations only
+            if (all_x) router_pieces();
         }
     }
     stamp(a, 2);
@@ -993,7 +1021,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int pr_lo = (int)((long long)(H / 2) * blockIdx.x / gridDim.x);  // one token: this CTA's output row pairs
     const int npr = (int)((long long)(H / 2) * (blockIdx.x + 1) / gridDim.x) - pr_lo;
     float* s_logit = reinterpret_cast<float*>(lsm + ls.logit);
-    const int npc = a.n_pieces == 0 ? gH.per_lane : a.n_pieces;
+    const int npc = a.n_pieces == 0 ? (gH.per_lane + kPieceChunks - 1) / kPieceChunks : a.n_pieces;
     // router scores of the tokens: sums of the per-piece partials (independent loads), into shared memory
     auto sum_pieces = [&]() {
         for (int i = threadIdx.x; i < T * E; i += kLayerThreads) {
@@ -1006,9 +1034,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         __syncthreads();
     };
     if constexpr (kOutRows) {
-        // The shared expert's down rows for this CTA's output rows need no routing: their first
-        // loads are issued, then (hook) the token is scored and routed by warp 0 while the other
-        // warps stage h of the shared expert; no warp streams while the route is taken.
+        // The shared expert's gate/up rows need no routing: this CTA's share of them (an even split)
+        // has its first loads issued, then (hook) the token is scored and routed while no warp
+        // streams; then the shared rows, then the routed experts' rows.
         auto route_hook = [&]() {
             // the token's router scores (sums of the pieces), sigmoids and selection keys
             uint32_t* s_key = reinterpret_cast<uint32_t*>(u.mask);  // the union's token masks are not used here
@@ -1056,35 +1084,28 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 }
                 if (lane == 0) reinterpret_cast<int*>(u.tmp)[0] = n_kept;
                 stamp(a, 12);
-            } else {
-                stage_vecs(a.h, 0, F, 1, P, nullptr, 1, hs + (size_t)k * hvs,
-                           hcorr + (size_t)k * gF.nch * 8, (int)threadIdx.x - 32, kLayerThreads - 32);
-                stamp(a, 13, 32);
             }
             __syncthreads();
         };
         {
+            const int s_lo = (int)((long long)F * blockIdx.x / gridDim.x);
+            const int s_hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
             auto rows_of = [&](int j, RowPair& r) {
-                const size_t row = (size_t)E * H + 2 * (pr_lo + j);
-                r.q0 = a.down_q + row * (F / 2);
-                r.q1 = r.q0 + F / 2;
-                r.s0 = a.down_s + row * (F / kGroup);
-                r.s1 = r.s0 + F / kGroup;
+                const size_t row = (size_t)E * F + j;
+                r.q0 = a.gate_q + row * (H / 2);
+                r.q1 = a.up_q + row * (H / 2);
+                r.s0 = a.gate_s + row * (H / kGroup);
+                r.s1 = a.up_s + row * (H / kGroup);
             };
             auto vecs_of = [&](int, VecSet<MT>& v) {
                 v.m = 1;
 #pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    v.vi[t] = k;
-                }
+                for (int t = 0; t < MT; ++t) v.vi[t] = 0;
             };
-            auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
-                const float y = warp_sum2(tot[0][0], tot[1][0]);  // lane 0: row 2 j, lane 16: row 2 j + 1
-                if ((lane & 15) == 0) ypart[(2 * j + (lane >> 4)) * S1 + k] = y;
-            };
-            const int first = warp;
-            const int nj = first < npr ? (npr - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of,
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) { gateup_finish(j, P, true, v, tot); };
+            const int first = s_lo + warp;
+            const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
+            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of,
                                        fin, route_hook);
         }
         stamp(a, 14);
@@ -1296,17 +1317,19 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 
     // ======================= phase C: down =======================
     if constexpr (kOutRows) {
-        // one token: this CTA's output row pairs of the k routed slots; the loads of
-        // the first rows are issued before the grid barrier (the weights do not
-        // depend on it), the routed h vectors are staged after it
+        // one token: this CTA's output row pairs of the kept routed experts and the shared expert;
+        // the loads of the first rows are issued before the grid barrier (the weights do not
+        // depend on it), the h vectors are staged after it
         const int S = S1;
-        // item j = (group g = j / npr: the g-th kept expert in ascending order, row pair)
+        // item j = (slot g = j / npr: the g-th kept expert in ascending order, the shared expert
+        // at g = n_kept; row pair)
         const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
-        const FastDiv div_pr(npr, (long long)npr * n_kept);
+        const int n_slots = n_kept + 1;
+        const FastDiv div_pr(npr, (long long)npr * n_slots);
         auto rows_of = [&](int j, RowPair& r) {
             const int slot = div_pr(j), pr = pr_lo + (j - slot * npr);
-            int e = u.gexp[slot];
-            if (!COLI_IN_BOUNDS(e >= 0 && e < E && 2 * pr + 1 < H, a.err)) e = 0;
+            int e = slot < n_kept ? u.gexp[slot] : E;
+            if (!COLI_IN_BOUNDS(e >= 0 && e <= E && 2 * pr + 1 < H, a.err)) e = 0;
             const size_t row = (size_t)e * H + 2 * pr;
             r.q0 = a.down_q + row * (F / 2);
             r.q1 = r.q0 + F / 2;
@@ -1323,17 +1346,25 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         };
         auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
             const int slot = div_pr(j), pl = j - slot * npr;
+            const int col = slot < n_kept ? slot : k;  // the shared expert's column is k
             const float y = warp_sum2(tot[0][0], tot[1][0]);  // lane 0: row 2 pl, lane 16: row 2 pl + 1
-            if ((lane & 15) == 0) ypart[(2 * pl + (lane >> 4)) * S + slot] = y;
+            if ((lane & 15) == 0) ypart[(2 * pl + (lane >> 4)) * S + col] = y;
         };
         auto hook = [&]() {
             grid_barrier(bar, deadline, a.err);
             stamp(a, 6);
-            stage_h(n_kept, 0);  // h of the g-th kept expert sits at position g
+            // h of the g-th kept expert sits at position g, the shared expert's at P (= k)
+            if (n_kept == P) {
+                stage_h(n_kept + 1, 0);
+            } else {
+                stage_h(n_kept, 0);
+                stage_vecs(a.h, 0, F, 1, P, nullptr, 1, hs + (size_t)n_kept * hvs, hcorr + (size_t)n_kept * gF.nch * 8,
+                           (int)threadIdx.x, kLayerThreads);
+            }
             __syncthreads();
             stamp(a, 7);
         };
-        const int total = npr * n_kept;
+        const int total = npr * n_slots;
         const int first = warp;
         const int nj = first < total ? (total - first + kLayerWarps - 1) / kLayerWarps : 0;
         stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin,
