@@ -1166,6 +1166,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 }
             }
         }
+        stamp(a, 11);
         for (int e = threadIdx.x; e < E; e += kLayerThreads) u.mask[e] = 0ull;
         __syncthreads();
         // union: token masks per expert, counts, offsets, stable positions
@@ -1206,6 +1207,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         }
         __syncthreads();
 
+        stamp(a, 12);
         // segments: [shared down groups (several tokens)] + routed gate/up groups
         const int n_sd = kOutRows ? 0 : n_sg;
         const int nseg = n_sd + n_rg;
@@ -1226,6 +1228,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         int lo, hi;
         seg_cta_range(st, lo, hi);
 
+        stamp(a, 13);
         // shared expert's down rows (several tokens), one run per shared group
         for (int s = 0; s < n_sd; ++s) {
             const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
@@ -1264,6 +1267,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin);
         }
 
+        stamp(a, 14);
         // routed gate/up: one run over all routed groups when every token is staged,
         // else one run per group (its tokens staged)
         const int r_lo = max(lo, st.ipre[n_sd]), r_hi = hi;
@@ -1313,7 +1317,10 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         }
     }
     stamp(a, 5);
-    if constexpr (!kOutRows) grid_barrier(bar, deadline, a.err);
+    if constexpr (!kOutRows) {
+        grid_barrier(bar, deadline, a.err);
+        stamp(a, 6);
+    }
 
     // ======================= phase C: down =======================
     if constexpr (kOutRows) {
@@ -1434,7 +1441,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
             stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin);
         }
+        stamp(a, 7);
         grid_barrier(bar, deadline, a.err);
+        stamp(a, 8);
 
         // ======================= phase D: combine =======================
         const int per_row = H / 4;
