@@ -463,7 +463,8 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
     layer_alg = float(np.mean((U + 1) * c.expert_bytes)) + c.E * c.H * 4 + c.E * 4 + x_bytes + out_bytes
     layer_gbs = layer_alg / (ms_per_step * 1e-3) / 1e9
     kname, kstage, kfile = DOMINANT[path]
-    traffic = traffic_from_profiles(kfile, c.name)
+    # the committed summaries are of the default kernel on the plain top-k routing
+    traffic = traffic_from_profiles(kfile, c.name) if not (top_p or act_int8) else None
     prefill = path == "prefill"
     if prefill:
         # dominant kernel: the gate/up grouped GEMM, 2 * (pairs + shared) * 2F * H flops

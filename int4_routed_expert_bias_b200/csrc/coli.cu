@@ -78,6 +78,11 @@ struct DeviceInfo {
     bool ready = false;
     int sms = 0;
     int smem_optin = 0;
+    // decode-kernel residency already checked on this device: (kernel, dynamic shared memory) pairs
+    static constexpr int kFitSlots = 64;
+    const void* fit_kern[kFitSlots] = {};
+    size_t fit_bytes[kFitSlots] = {};
+    int n_fit = 0;
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -532,10 +537,12 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
 
     DeviceInfo* dev = nullptr;
     if ((st = device_info(&dev)) != COLI_OK) return st;
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    cudaError_t e = cudaStreamIsCapturing(stream, &cs);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
-    tm.capturing = (cs == cudaStreamCaptureStatusActive);
+    cudaError_t e = cudaSuccess;
+    if (tm.ev) {  // stage events requested (test hook): recorded differently inside a graph capture
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if ((e = cudaStreamIsCapturing(stream, &cs)) != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+        tm.capturing = (cs == cudaStreamCaptureStatusActive);
+    }
     tm.s = stream;
 
     int32_t* idx = topk_idx_out ? topk_idx_out : w.idx;
@@ -552,10 +559,29 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
         const LayerPlan pl = layer_plan(T, H, F, E, k);
         if (dev->sms < kMinLayerSms) return fail(COLI_ERR_UNSUPPORTED, "%d SMs: the decode kernel needs %d", dev->sms, kMinLayerSms);
         const LayerKernel kern = layer_kernel(pl.MT, bf16, ot == COLI_BF16, pl.out_rows, L->act_int8 != 0);
-        int occ = 0;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, layer_threads(pl.MT), pl.ls.bytes)) != cudaSuccess)
-            return cuda_fail(e, "occupancy query");
-        if (occ < 1) return fail(COLI_ERR_UNSUPPORTED, "the decode kernel does not fit on an SM (%zu B shared memory)", pl.ls.bytes);
+        {  // one block per SM must be resident (a cooperative launch); the answer is cached per (kernel, bytes)
+            bool known = false;
+            {
+                std::lock_guard<std::mutex> lock(g_dev_mu);
+                for (int i = 0; i < dev->n_fit && !known; ++i)
+                    known = dev->fit_kern[i] == (const void*)kern && dev->fit_bytes[i] == pl.ls.bytes;
+            }
+            if (!known) {
+                int occ = 0;
+                if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, layer_threads(pl.MT), pl.ls.bytes)) !=
+                    cudaSuccess)
+                    return cuda_fail(e, "occupancy query");
+                if (occ < 1)
+                    return fail(COLI_ERR_UNSUPPORTED, "the decode kernel does not fit on an SM (%zu B shared memory)",
+                                pl.ls.bytes);
+                std::lock_guard<std::mutex> lock(g_dev_mu);
+                if (dev->n_fit < DeviceInfo::kFitSlots) {
+                    dev->fit_kern[dev->n_fit] = (const void*)kern;
+                    dev->fit_bytes[dev->n_fit] = pl.ls.bytes;
+                    ++dev->n_fit;
+                }
+            }
+        }
         const bool fused_router = T <= pl.MT;
         if ((e = tm.rec(COLI_STAGE_ROUTE, 0)) != cudaSuccess) return cuda_fail(e, "event record");
         if (!fused_router) {
