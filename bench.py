@@ -329,15 +329,18 @@ class Resident:
         self.H, self.F, self.E = c.H, c.F, c.E
 
 
-def path_dtype(path, act_int8=False):
+def path_dtype(path, act_int8=False, x_bf16=False):
     """Arithmetic the timed path computes in: the tensor-core prefill in bf16
     operands with fp32 accumulation; the decode kernel in exact int32 products
-    of int4 weights and fixed-point (21-bit, or int8 for the variant)
-    activations, accumulated in fp32; the CUDA-core wide path in fp32."""
+    of int4 weights and fixed-point activations (21-bit for fp32 inputs,
+    15-bit for bf16 inputs, int8 for the variant), accumulated in fp32; the
+    CUDA-core wide path in fp32."""
     if path == "prefill":
         return "bf16"
     if path in ("single", "decode"):
-        return "int8xint4->int32/f32" if act_int8 else "int32/f32"
+        if act_int8:
+            return "int8xint4->int32/f32"
+        return "fx15xint4->int32/f32" if x_bf16 else "fx21xint4->int32/f32"
     return "f32"
 
 
@@ -501,7 +504,7 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
     entry = {"workload": workload_desc(c) + (f", adaptive expert top-p {top_p}" if top_p else "") +
              (", int8 activations (integer-dot variant)" if act_int8 else ""),
              "tokens_per_call": c.T, "path": path, "value": value, "top_p": top_p, "act_int8": bool(act_int8),
-             "dtype": path_dtype(path, act_int8),
+             "dtype": path_dtype(path, act_int8, c.x_dtype == "bf16"),
              "unit": "tokens/s", "steps": steps, "timed_replays": R, "ms_per_step": ms_per_step,
              "ms_per_step_p10": percentile(ms_max, 10) / steps, "ms_per_step_p90": percentile(ms_max, 90) / steps,
              "roofline": roofline, "gpu_launches": steps * kernels_per_call(path, c.T, c.E),

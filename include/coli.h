@@ -148,10 +148,12 @@ COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
  * no expert reads.  The rule is this library's reading: the page names the
  * knob and its effect only.  The router is fp32.  Batches of up to 64 tokens
  * compute the experts with fp32 accumulation; the activations (and the SwiGLU
- * output h) enter the expert products as 21-bit fixed point per block of 32
- * values (power-of-two block scale; each value within 2^-21 of its block's
- * largest magnitude), multiplied exactly in integers: an error of the order of
- * fp32 arithmetic.  Larger batches run the experts on the tensor cores with
+ * output h) enter the expert products as fixed point per block of 32 values
+ * over a power-of-two block scale, multiplied exactly in integers: 21 bits for
+ * fp32 activations (each value within 2^-21 of its block's largest magnitude,
+ * an error of the order of fp32 arithmetic), 14 bits plus sign for bf16
+ * activations (within 2^-15 of the block's largest magnitude, well below the
+ * up to 2^-9 relative rounding the bf16 inputs carry).  Larger batches run the experts on the tensor cores with
  * bf16 operands (weights q * scale, activations and the SwiGLU output rounded
  * to bf16) and fp32 accumulation.
  * Integer-activation variant (layer->act_int8 = 1; "Colibri 完全ガイド", section

@@ -379,6 +379,88 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
     }
 }
 
+// Two-digit staging for bf16 activations: 14-bit fixed point plus sign over the
+// chunk's power-of-two scale, X = round(x * 2^(14 - e)) held at 2^14 - 1, as
+// X = 128 d0 + d1 (d0 the signed top byte, d1 seven unsigned bits) in the
+// first two plane pairs, and a float2 (2^(e - 14), 8 * sum X) per chunk.  The
+// rounding error, at most 2^-15 m per value, stays far below the bf16 rounding
+// (up to 2^-9 |x|) that the activations already carry, and it takes two dp4a
+// planes instead of three.  Chunk rules as in stage_rows_digits.
+static __device__ __noinline__ void stage_rows_digits2(const void* __restrict__ src, int bf16, int K, int n, int row0,
+                                                       const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
+                                                       int nthr)
+{
+    const int nch = K / kChunkK;
+    const int vunits = digit_vec_units(K);
+    const size_t row_bytes = (size_t)K * (bf16 ? 2 : 4);
+    for (int idx = tid; idx < n * nch; idx += nthr) {
+        const int t = idx / nch, c = idx - t * nch;
+        const int row = tbl ? tbl[t] / tdiv : row0 + t;
+        const char* rp = static_cast<const char*>(src) + (size_t)row * row_bytes;
+        float x[32];
+        if (bf16) {
+            const uint4* p4 = reinterpret_cast<const uint4*>(rp + (size_t)c * kChunkK * 2);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v = p4[j];
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    x[8 * j + 2 * h] = bf16_bits_to_float(u[h] & 0xFFFFu);
+                    x[8 * j + 2 * h + 1] = bf16_bits_to_float(u[h] >> 16);
+                }
+            }
+        } else {
+            const float4* p4 = reinterpret_cast<const float4*>(rp + (size_t)c * kChunkK * 4);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 v = p4[j];
+                x[4 * j] = v.x;
+                x[4 * j + 1] = v.y;
+                x[4 * j + 2] = v.z;
+                x[4 * j + 3] = v.w;
+            }
+        }
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(x[j]));
+        const bool finite = m <= 3.402823466e38f;  // false for inf and NaN
+        const int ex = (int)(__float_as_uint(m) >> 23);
+        const bool live = finite && ex >= 26;  // m >= 2^-100, as in stage_rows_digits
+        const int e = live ? ex - 126 : 0;     // m < 2^e
+        const float mult = live ? __uint_as_float((uint32_t)(141 - e) << 23) : 0.f;  // 2^(14 - e)
+        uint32_t X[32];
+        int csum = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int v = __float_as_int(fmaf(x[j], mult, 12582912.0f)) - 0x4B400000;
+            const int vc = min(v, (1 << 14) - 1);
+            X[j] = (uint32_t)vc;
+            csum += vc;
+        }
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
+        uint32_t lo[4], hi[4];
+        // plane d1: bits 0-6; d0: bits 7-14 (signed)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            lo[w] = pack_lo_bytes(X[8 * w], X[8 * w + 2], X[8 * w + 4], X[8 * w + 6]) & 0x7F7F7F7Fu;
+            hi[w] = pack_lo_bytes(X[8 * w + 1], X[8 * w + 3], X[8 * w + 5], X[8 * w + 7]) & 0x7F7F7F7Fu;
+        }
+        base[2 * 32] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        base[3 * 32] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            lo[w] = pack_lo_bytes(X[8 * w] >> 7, X[8 * w + 2] >> 7, X[8 * w + 4] >> 7, X[8 * w + 6] >> 7);
+            hi[w] = pack_lo_bytes(X[8 * w + 1] >> 7, X[8 * w + 3] >> 7, X[8 * w + 5] >> 7, X[8 * w + 7] >> 7);
+        }
+        base[0 * 32] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        base[1 * 32] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        const float scale = !finite ? __int_as_float(0x7FC00000) : live ? __uint_as_float((uint32_t)(113 + e) << 23)
+                                                                          : 0.f;
+        xc[(size_t)t * nch + c] = make_float2(scale, __int_as_float(8 * csum));
+    }
+}
+
 // The integer-activation variant's staging: one plane pair of symmetric int8
 // codes per chunk, code = rint(x * (127 / m)) with m = max |x| of the chunk,
 // scale m / 127 (a chunk whose 127 / m overflows fp32 is zero; one holding inf

@@ -166,9 +166,12 @@ __device__ __forceinline__ void chunk_pair_digit_vectors(const uint4& w0, const 
             const float2 c = cc[v.vi[t] * nch];
             const uint32_t corr = (uint32_t)__float_as_int(c.y);
             uint32_t D0 = (uint32_t)a0[0], D1 = (uint32_t)a1[0];
-            if (nd == 3) {  // X = 16384 d0 + 128 d1 + d2; one plane: X = d0
+            if (nd == 3) {  // X = 16384 d0 + 128 d1 + d2; two planes: 128 d0 + d1; one plane: X = d0
                 D0 = (D0 * 128u + (uint32_t)a0[1]) * 128u + (uint32_t)a0[2];
                 D1 = (D1 * 128u + (uint32_t)a1[1]) * 128u + (uint32_t)a1[2];
+            } else if (nd == 2) {
+                D0 = D0 * 128u + (uint32_t)a0[1];
+                D1 = D1 * 128u + (uint32_t)a1[1];
             }
             D0 -= corr;
             D1 -= corr;
@@ -852,7 +855,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
-    constexpr int nd = kI8 ? 1 : 3;  // digit planes per staged vector (int8 variant: one)
+    // digit planes per staged vector: fp32 activations three (21-bit), bf16 two (14-bit), the int8 variant one
+    constexpr int nd = kI8 ? 1 : kBf16 ? 2 : 3;
     constexpr int kPieceChunks = MT == 1 ? 2 : 1;  // router chunks per lane per piece
     // staged vectors as digit planes (16-byte units per vector)
     const int xvs = digit_vec_units(H);
@@ -882,6 +886,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         if constexpr (kI8)
             stage_rows_int8(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
                             reinterpret_cast<float2*>(dcorr), tid, nthr);
+        else if constexpr (kBf16)
+            stage_rows_digits2(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
+                               reinterpret_cast<float2*>(dcorr), tid, nthr);
         else
             stage_rows_digits(src, bf16, K, n, row0, tbl, tdiv, reinterpret_cast<uint4*>(dst),
                               reinterpret_cast<float2*>(dcorr), tid, nthr);
