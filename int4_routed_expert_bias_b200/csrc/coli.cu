@@ -394,13 +394,14 @@ struct LayerPlan {
     LayerSmem ls{};
 };
 
-LayerPlan layer_plan(int T, int H, int F, int E, int k)
+// nd: digits per staged activation (3: fp32 activations, 2: bf16, 1: the int8 variant).
+LayerPlan layer_plan(int T, int H, int F, int E, int k, int nd)
 {
     LayerPlan p;
     if (T < 1 || T > kLayerMaxT) return p;
     const int rows_per_cta = 2 * ((H / 2 + kMinLayerSms - 1) / kMinLayerSms);
     auto fits = [&](int MT, bool rows) {
-        const LayerSmem ls = layer_smem(T, H, F, E, k, MT, rows, rows_per_cta);
+        const LayerSmem ls = layer_smem(T, H, F, E, k, MT, rows, rows_per_cta, nd);
         if (ls.bytes > (size_t)kSmemBudget) return false;
         p.ok = true;
         p.MT = MT;
@@ -420,7 +421,8 @@ int choose_path(const coli_moe_layer* L, int T)
 {
     if (T == 0) return COLI_PATH_NONE;
     if (T <= kDecodeMaxT) {
-        const LayerPlan pl = layer_plan(T, L->hidden, L->ffn, L->n_experts, L->top_k);
+        // the path does not depend on the activations' type: plan with the largest staging (fp32)
+        const LayerPlan pl = layer_plan(T, L->hidden, L->ffn, L->n_experts, L->top_k, L->act_int8 ? 1 : 3);
         if (pl.ok) return pl.out_rows ? COLI_PATH_SINGLE : COLI_PATH_DECODE;
     }
     if (T > kDecodeMaxT && L->hidden % kPfRawK == 0 && L->ffn % kPfRawK == 0) return COLI_PATH_PREFILL;
@@ -556,7 +558,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
     // Up to 64 tokens: the fused decode-layer kernel, one cooperative launch
     // (after the router-score kernel when the batch is larger than one token group).
     if (path == COLI_PATH_SINGLE || path == COLI_PATH_DECODE) {
-        const LayerPlan pl = layer_plan(T, H, F, E, k);
+        const LayerPlan pl = layer_plan(T, H, F, E, k, L->act_int8 ? 1 : bf16 ? 2 : 3);
         if (dev->sms < kMinLayerSms) return fail(COLI_ERR_UNSUPPORTED, "%d SMs: the decode kernel needs %d", dev->sms, kMinLayerSms);
         const LayerKernel kern = layer_kernel(pl.MT, bf16, ot == COLI_BF16, pl.out_rows, L->act_int8 != 0);
         {  // one block per SM must be resident (a cooperative launch); the answer is cached per (kernel, bytes)

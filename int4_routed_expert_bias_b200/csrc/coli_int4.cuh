@@ -249,21 +249,21 @@ static __device__ __noinline__ void stage_rows(const void* __restrict__ src, int
 // only: d0 = round(x * 127 / m), scale m / 127 (the pages' integer dot-product
 // kernel, "Colibri 完全ガイド", section コア技術のハイライト).
 //
-// Shared-memory layout of one staged vector: chunk c = l + 32 i, plane
-// p = 2 * digit + (0: lo, 1: hi), as uint4 at ((i * 6 + p) * 32 + l); word w
-// of the uint4 covers k = 8 w .. 8 w + 7 of the chunk, byte b of a lo (hi)
-// word holds the digit of k = 8 w + 2 b (+ 1).  Per chunk one float2:
-// (2^(e - 21), corr as int bits).
-constexpr int kDigitPlanes = 6;
+// Shared-memory layout of one staged vector with nd digits (np = 2 nd planes):
+// chunk c = l + 32 i, plane p = 2 * digit + (0: lo, 1: hi), as uint4 at
+// ((i * np + p) * 32 + l); word w of the uint4 covers k = 8 w .. 8 w + 7 of
+// the chunk, byte b of a lo (hi) word holds the digit of k = 8 w + 2 b (+ 1).
+// Per chunk one float2: (2^(e - 21), corr as int bits).
+__host__ __device__ constexpr int digit_planes(int nd) { return 2 * nd; }
 
-__host__ __device__ inline int digit_vec_units(int K)  // 16-byte units per staged vector
+__host__ __device__ inline int digit_vec_units(int K, int nd)  // 16-byte units per staged vector
 {
-    return stage_geom(K).per_lane * kDigitPlanes * 32;
+    return stage_geom(K).per_lane * digit_planes(nd) * 32;
 }
 
-__host__ __device__ inline size_t digit_smem_bytes(int K, int n_vectors)
+__host__ __device__ inline size_t digit_smem_bytes(int K, int n_vectors, int nd)
 {
-    return (size_t)n_vectors * digit_vec_units(K) * 16 + (size_t)n_vectors * (K / kChunkK) * 8;
+    return (size_t)n_vectors * digit_vec_units(K, nd) * 16 + (size_t)n_vectors * (K / kChunkK) * 8;
 }
 
 // biased bytes q + 8 of nibbles 0, 2, 4, 6 (lo) and 1, 3, 5, 7 (hi) of a word
@@ -297,8 +297,9 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
                                                       const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
                                                       int nthr)
 {
+    constexpr int ND = 3;  // digits per value
     const int nch = K / kChunkK;
-    const int vunits = digit_vec_units(K);
+    const int vunits = digit_vec_units(K, ND);
     const size_t row_bytes = (size_t)K * (bf16 ? 2 : 4);
     for (int idx = tid; idx < n * nch; idx += nthr) {
         const int t = idx / nch, c = idx - t * nch;
@@ -348,7 +349,7 @@ static __device__ __noinline__ void stage_rows_digits(const void* __restrict__ s
             X[j] = (uint32_t)vc;
             csum += vc;
         }
-        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * digit_planes(ND) * 32 + (c & 31);
         uint32_t lo[4], hi[4];
         // plane d2: bits 0-6; d1: bits 7-13; d0: bits 14-21 (signed)
 #pragma unroll
@@ -390,8 +391,9 @@ static __device__ __noinline__ void stage_rows_digits2(const void* __restrict__ 
                                                        const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
                                                        int nthr)
 {
+    constexpr int ND = 2;  // digits per value
     const int nch = K / kChunkK;
-    const int vunits = digit_vec_units(K);
+    const int vunits = digit_vec_units(K, ND);
     const size_t row_bytes = (size_t)K * (bf16 ? 2 : 4);
     for (int idx = tid; idx < n * nch; idx += nthr) {
         const int t = idx / nch, c = idx - t * nch;
@@ -438,7 +440,7 @@ static __device__ __noinline__ void stage_rows_digits2(const void* __restrict__ 
             X[j] = (uint32_t)vc;
             csum += vc;
         }
-        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * digit_planes(ND) * 32 + (c & 31);
         uint32_t lo[4], hi[4];
         // plane d1: bits 0-6; d0: bits 7-14 (signed)
 #pragma unroll
@@ -470,8 +472,9 @@ static __device__ __noinline__ void stage_rows_int8(const void* __restrict__ src
                                                     const int* tbl, int tdiv, uint4* xd, float2* xc, int tid,
                                                     int nthr)
 {
+    constexpr int ND = 1;  // digits per value
     const int nch = K / kChunkK;
-    const int vunits = digit_vec_units(K);
+    const int vunits = digit_vec_units(K, ND);
     const size_t row_bytes = (size_t)K * (bf16 ? 2 : 4);
     for (int idx = tid; idx < n * nch; idx += nthr) {
         const int t = idx / nch, c = idx - t * nch;
@@ -515,7 +518,7 @@ static __device__ __noinline__ void stage_rows_int8(const void* __restrict__ src
             X[j] = (uint32_t)v;
             csum += v;
         }
-        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * kDigitPlanes * 32 + (c & 31);
+        uint4* base = xd + (size_t)t * vunits + (size_t)(c >> 5) * digit_planes(ND) * 32 + (c & 31);
         uint32_t lo[4], hi[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {

@@ -107,12 +107,11 @@ __device__ __forceinline__ void grid_barrier(GridBar& b, unsigned long long dead
 // ---------------------------------------------------------------------------
 // the rolling int4 row-pair engine
 
-// Two int4 rows (bytes and scales) that one item streams.
-struct RowPair {
-    const uint8_t* q0;
-    const uint8_t* q1;
-    const float* s0;
-    const float* s1;
+// The int4 rows (bytes and scales) that one item streams, RW of them.
+template <int RW>
+struct Rows {
+    const uint8_t* q[RW];
+    const float* s[RW];
 };
 
 // The staged vectors that one item multiplies its rows with (indices into the
@@ -124,79 +123,70 @@ struct VecSet {
     int vi[MT];  // staged-vector index of vector t
 };
 
-// One 16-byte chunk of both rows against up to MT digit-staged vectors (see
-// coli_int4.cuh): each word of each row is decoded once into biased bytes and
-// applied to every vector with dp4a.  xd = this lane's plane 0 of the chunk in
-// vector 0's frame; cc = this lane's chunk entry in vector 0's frame.
-template <int MT>
-__device__ __forceinline__ void chunk_pair_digit_vectors(const uint4& w0, const uint4& w1, const uint4* xd,
-                                                         const float2* cc, const VecSet<MT>& v, int vstride, int nch,
-                                                         int nd, float s0, float s1, float (&tot)[2][MT])
+// One 16-byte chunk of each of the RW rows against up to MT digit-staged
+// vectors of ND digits (see coli_int4.cuh): each word of each row is decoded
+// once into biased bytes and applied to every vector with dp4a; every
+// activation load serves all RW rows.  xd = this lane's plane 0 of the chunk
+// in vector 0's frame; cc = this lane's chunk entry in vector 0's frame.
+template <int MT, int RW, int ND>
+__device__ __forceinline__ void chunk_rows_digit_vectors(const uint4 (&w)[RW], const uint4* xd, const float2* cc,
+                                                         const VecSet<MT>& v, int vstride, int nch,
+                                                         const float (&sc)[RW], float (&tot)[RW][MT])
 {
-    uint32_t al[4], ah[4], bl[4], bh[4];
+    uint32_t lo[RW][4], hi[RW][4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t a = q == 0 ? w0.x : q == 1 ? w0.y : q == 2 ? w0.z : w0.w;
-        const uint32_t b = q == 0 ? w1.x : q == 1 ? w1.y : q == 2 ? w1.z : w1.w;
-        al[q] = nib_lo_u8(a);
-        ah[q] = nib_hi_u8(a);
-        bl[q] = nib_lo_u8(b);
-        bh[q] = nib_hi_u8(b);
+    for (int r = 0; r < RW; ++r) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t a = q == 0 ? w[r].x : q == 1 ? w[r].y : q == 2 ? w[r].z : w[r].w;
+            lo[r][q] = nib_lo_u8(a);
+            hi[r][q] = nib_hi_u8(a);
+        }
     }
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
         if (t < v.m) {
             const uint4* x = xd + v.vi[t] * vstride;
-            int a0[3] = {0, 0, 0}, a1[3] = {0, 0, 0};
+            int acc[RW][ND];
 #pragma unroll
-            for (int d = 0; d < 3; ++d) {
-                if (d < nd) {
-                    const uint4 xl = x[(2 * d) * 32], xh = x[(2 * d + 1) * 32];
+            for (int r = 0; r < RW; ++r)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t l = q == 0 ? xl.x : q == 1 ? xl.y : q == 2 ? xl.z : xl.w;
-                        const uint32_t h = q == 0 ? xh.x : q == 1 ? xh.y : q == 2 ? xh.z : xh.w;
-                        a0[d] = dp4a_us(al[q], l, a0[d]);
-                        a0[d] = dp4a_us(ah[q], h, a0[d]);
-                        a1[d] = dp4a_us(bl[q], l, a1[d]);
-                        a1[d] = dp4a_us(bh[q], h, a1[d]);
+                for (int d = 0; d < ND; ++d) acc[r][d] = 0;
+#pragma unroll
+            for (int d = 0; d < ND; ++d) {
+                const uint4 xl = x[(2 * d) * 32], xh = x[(2 * d + 1) * 32];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t l = q == 0 ? xl.x : q == 1 ? xl.y : q == 2 ? xl.z : xl.w;
+                    const uint32_t h = q == 0 ? xh.x : q == 1 ? xh.y : q == 2 ? xh.z : xh.w;
+#pragma unroll
+                    for (int r = 0; r < RW; ++r) {
+                        acc[r][d] = dp4a_us(lo[r][q], l, acc[r][d]);
+                        acc[r][d] = dp4a_us(hi[r][q], h, acc[r][d]);
                     }
                 }
             }
             const float2 c = cc[v.vi[t] * nch];
             const uint32_t corr = (uint32_t)__float_as_int(c.y);
-            uint32_t D0 = (uint32_t)a0[0], D1 = (uint32_t)a1[0];
-            if (nd == 3) {  // X = 16384 d0 + 128 d1 + d2; two planes: 128 d0 + d1; one plane: X = d0
-                D0 = (D0 * 128u + (uint32_t)a0[1]) * 128u + (uint32_t)a0[2];
-                D1 = (D1 * 128u + (uint32_t)a1[1]) * 128u + (uint32_t)a1[2];
-            } else if (nd == 2) {
-                D0 = D0 * 128u + (uint32_t)a0[1];
-                D1 = D1 * 128u + (uint32_t)a1[1];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                // X = 16384 d0 + 128 d1 + d2 (three digits), 128 d0 + d1 (two), d0 (one)
+                uint32_t D = (uint32_t)acc[r][0];
+#pragma unroll
+                for (int d = 1; d < ND; ++d) D = D * 128u + (uint32_t)acc[r][d];
+                D -= corr;
+                tot[r][t] = fmaf(sc[r] * c.x, (float)(int)D, tot[r][t]);
             }
-            D0 -= corr;
-            D1 -= corr;
-            tot[0][t] = fmaf(s0 * c.x, (float)(int)D0, tot[0][t]);
-            tot[1][t] = fmaf(s1 * c.x, (float)(int)D1, tot[1][t]);
         }
     }
 }
 
-// Streams items j0, j0 + js, ... (nj of them) of a row-pair list: item j has
-// two int4 rows of K = 32 * nch values (rows_of(j, RowPair&)) and up to MT
-// staged vectors (vecs_of(j, VecSet&)).  The lane takes chunks c = lane + 32 i,
-// i < per_lane; a step is one chunk of both rows (16 bytes of each and their
-// two scales).  The steps' bytes travel through this warp's ring of R slots in
-// shared memory, filled by cp.async R - 1 steps ahead of the one being
-// computed, so the bytes in flight do not cost registers and the loop stays
-// small (the slot index is an address, not a register name).  At the end of
-// item j, finish(j, VecSet, tot) gets the lane's partial sums tot[row][vector]
-// (to be summed over the warp).  xs: staged float4 slots; corr: staged chunk
-// corrections; ring: this warp's R * kSlotBytes bytes.
 struct NoHook {
     __device__ void operator()() const {}
 };
 
-constexpr int kSlotBytes = 32 * (16 + 16 + 4 + 4);  // one step of a warp: two 16-byte chunks and two scales per lane
+// Bytes of one ring slot (one step of a warp): RW 16-byte chunks and RW scales per lane.
+__host__ __device__ constexpr int slot_bytes(int RW) { return 32 * RW * (16 + 4); }
 
 // hook(): called by every thread once the first R - 1 steps are in flight and
 // before the first one is consumed (e.g. a barrier and the staging of the
@@ -242,49 +232,63 @@ __device__ __forceinline__ float lds32(uint32_t smem)
     return r;
 }
 
-template <int MT, int R, typename RowsOf, typename VecsOf, typename Finish, typename Hook = NoHook>
-__device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per_lane, int nch, const float4* xs,
-                                                 const void* corr, int nd, unsigned char* ring, RowsOf rows_of,
-                                                 VecsOf vecs_of, Finish finish, Hook hook = Hook())
+// Streams items j0, j0 + js, ... (nj of them) of a row list: item j has RW
+// int4 rows of K = 32 * nch values (rows_of(j, Rows<RW>&)) and up to MT staged
+// vectors of ND digits (vecs_of(j, VecSet&)).  The lane takes chunks
+// c = lane + 32 i, i < per_lane; a step is one chunk of every row (16 bytes of
+// each and their scales).  The steps' bytes travel through this warp's ring of
+// R slots in shared memory, filled by cp.async R - 1 steps ahead of the one
+// being computed, so the bytes in flight do not cost registers and the loop
+// stays small (the slot index is an address, not a register name).  At the
+// end of item j, finish(j, VecSet, tot) gets the lane's partial sums
+// tot[row][vector] (to be summed over the warp).  xs: staged digit planes;
+// corr: staged chunk entries; ring: this warp's R * slot_bytes(RW) bytes.
+template <int MT, int RW, int R, int ND, typename RowsOf, typename VecsOf, typename Finish, typename Hook = NoHook>
+__device__ __forceinline__ void stream_rows(int j0, int js, int nj, int per_lane, int nch, const float4* xs,
+                                            const void* corr, unsigned char* ring, RowsOf rows_of, VecsOf vecs_of,
+                                            Finish finish, Hook hook = Hook())
 {
     if (nj <= 0) {
         hook();
         return;
     }
+    constexpr uint32_t kSlot = slot_bytes(RW);
     const int lane = threadIdx.x & 31;
     const bool whole = (nch & 31) == 0;  // every lane has a chunk at every step
-    // this lane's bytes of ring slot 0 (16-byte chunk of row 0 at +0, of row 1 at +512; scales at sc_off, +128)
+    // this lane's bytes of ring slot 0: the 16-byte chunk of row r at +512 r, its scale at sc_off + 128 r
     const uint32_t ring_lane = smem_u32(ring) + lane * 16;
-    const uint32_t ring_end = ring_lane + R * kSlotBytes;
-    const uint32_t sc_off = 1024 - 12 * lane;
+    const uint32_t ring_end = ring_lane + R * kSlot;
+    const uint32_t sc_off = 512 * RW - 12 * lane;
     const uint64_t pol = l2_evict_first();
     // load cursor: item lj (0-based among mine), chunk step lci, this lane's slot address and source pointers
     int lj = 0, lci = 0;
     uint32_t lsl = ring_lane;
-    const uint8_t *pq0, *pq1;
-    const float *ps0, *ps1;
+    const uint8_t* pq[RW];
+    const float* ps[RW];
     auto set_rows = [&](int j) {
-        RowPair r;
+        Rows<RW> r;
         rows_of(j, r);
-        pq0 = r.q0 + lane * 16;
-        pq1 = r.q1 + lane * 16;
-        ps0 = r.s0 + (lane >> 1);
-        ps1 = r.s1 + (lane >> 1);
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+            pq[i] = r.q[i] + lane * 16;
+            ps[i] = r.s[i] + (lane >> 1);
+        }
     };
     set_rows(j0);
     auto issue = [&]() {
         if (lj < nj && (whole || lane + 32 * lci < nch)) {
-            cp_async16_s(lsl, pq0, pol);
-            cp_async16_s(lsl + 512, pq1, pol);
-            cp_async4_s(lsl + sc_off, ps0, pol);
-            cp_async4_s(lsl + sc_off + 128, ps1, pol);
+#pragma unroll
+            for (int i = 0; i < RW; ++i) cp_async16_s(lsl + 512 * i, pq[i], pol);
+#pragma unroll
+            for (int i = 0; i < RW; ++i) cp_async4_s(lsl + sc_off + 128 * i, ps[i], pol);
         }
         cp_async_commit();  // one group per step (empty past the end)
-        pq0 += 512;         // this lane's next chunk: 32 chunks on
-        pq1 += 512;
-        ps0 += 16;
-        ps1 += 16;
-        lsl += kSlotBytes;
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+            pq[i] += 512;  // this lane's next chunk: 32 chunks on
+            ps[i] += 16;
+        }
+        lsl += kSlot;
         if (lsl == ring_end) lsl = ring_lane;
         if (++lci == per_lane) {
             lci = 0;
@@ -299,11 +303,13 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
     uint32_t csl = ring_lane;
     VecSet<MT> v;
     vecs_of(j0, v);
-    float tot[2][MT];
+    float tot[RW][MT];
 #pragma unroll
-    for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
-    // staged vectors: digit planes, 6 x 32 units of 16 bytes per chunk step; a float2 entry per chunk
-    constexpr int kXStep = kDigitPlanes * 32;
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int t = 0; t < MT; ++t) tot[r][t] = 0.f;
+    // staged vectors: 2 ND planes of 32 units of 16 bytes per chunk step; a float2 entry per chunk
+    constexpr int kXStep = digit_planes(ND) * 32;
     const int vstride = per_lane * kXStep;  // 16-byte units per staged vector
     const uint4* xrow = reinterpret_cast<const uint4*>(xs) + lane;
     const float2* crow = static_cast<const float2*>(corr) + lane;
@@ -313,11 +319,16 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
         issue();                   // step s + R - 1 into the slot consumed last iteration
         cp_async_wait<R - 1>();    // step s has landed (this lane's own bytes)
         if (whole || lane + 32 * cci < nch) {
-            const uint4 w0 = lds128(csl), w1 = lds128(csl + 512);
-            const float s0 = lds32(csl + sc_off), s1 = lds32(csl + sc_off + 128);
-            chunk_pair_digit_vectors<MT>(w0, w1, xrow, crow, v, vstride, nch, nd, s0, s1, tot);
+            uint4 w[RW];
+            float sc[RW];
+#pragma unroll
+            for (int i = 0; i < RW; ++i) {
+                w[i] = lds128(csl + 512 * i);
+                sc[i] = lds32(csl + sc_off + 128 * i);
+            }
+            chunk_rows_digit_vectors<MT, RW, ND>(w, xrow, crow, v, vstride, nch, sc, tot);
         }
-        csl += kSlotBytes;
+        csl += kSlot;
         if (csl == ring_end) csl = ring_lane;
         xrow += kXStep;
         crow += 32;
@@ -327,7 +338,9 @@ __device__ __forceinline__ void stream_row_pairs(int j0, int js, int nj, int per
             crow = static_cast<const float2*>(corr) + lane;
             finish(j0 + cj * js, v, tot);
 #pragma unroll
-            for (int t = 0; t < MT; ++t) tot[0][t] = tot[1][t] = 0.f;
+            for (int r = 0; r < RW; ++r)
+#pragma unroll
+                for (int t = 0; t < MT; ++t) tot[r][t] = 0.f;
             if (++cj < nj) vecs_of(j0 + cj * js, v);
         }
     }
@@ -380,25 +393,35 @@ struct LayerSmem {
     // union tables (byte offsets from the start of shared memory)
     uint32_t mask, cnt, off, gpre, idx, w, perm, ipos, gexp, gpos, seg_c, seg_i, seg_cost, tmp;
     uint32_t logit;  // router scores [T, E] of the tokens (when the kernel scores them itself)
-    uint32_t ring;   // the warps' cp.async rings, warps x ring_slots x kSlotBytes
+    uint32_t ring;   // the warps' cp.async rings, warps x ring_slots x slot_bytes(layer_rows(MT, nd))
     int ring_slots;
 };
 
-// Ring slots per warp: deeper when fewer activation vectors are staged.
-__host__ __device__ constexpr int layer_ring_slots(int MT) { return MT == 1 ? 5 : 4; }
+// Rows per engine step: four for groups of several tokens whose activations
+// take at most two digits (each activation load then serves four rows; their
+// ring fits beside the staged vectors), else two.
+__host__ __device__ constexpr int layer_rows(int MT, int nd) { return MT > 1 && nd <= 2 ? 4 : 2; }
 
-// rows_per_cta: output rows of one CTA in the one-token output-row mode.
+// Ring slots per warp (steps in flight + 1): deeper when fewer activation
+// vectors are staged, shallower for the four-row slots.
+__host__ __device__ constexpr int layer_ring_slots(int MT, int nd)
+{
+    return layer_rows(MT, nd) == 4 ? 3 : MT == 1 ? 5 : 4;
+}
+
+// rows_per_cta: output rows of one CTA in the one-token output-row mode; nd:
+// digits per staged activation (3 for fp32 inputs, 2 for bf16, 1 for int8).
 __host__ __device__ inline LayerSmem layer_smem(int T, int H, int F, int E, int k, int MT, bool out_rows,
-                                                int rows_per_cta)
+                                                int rows_per_cta, int nd)
 {
     LayerSmem s{};
     s.nx = T <= MT ? T : MT;
     s.nh = out_rows ? k + 1 : MT;
     size_t off = 0;
     s.x_off = off;
-    off += align_up(digit_smem_bytes(H, s.nx), 16);
+    off += align_up(digit_smem_bytes(H, s.nx, nd), 16);
     s.h_off = off;
-    off += align_up(digit_smem_bytes(F, s.nh), 16);
+    off += align_up(digit_smem_bytes(F, s.nh, nd), 16);
     s.u_off = off;
     {
         const size_t P = (size_t)T * k;
@@ -423,8 +446,8 @@ __host__ __device__ inline LayerSmem layer_smem(int T, int H, int F, int E, int 
         s.seg_cost = take((P + (size_t)E + 70) * 4);
         s.tmp = take(32 * 8);
         s.logit = take(T <= MT ? (size_t)T * E * 4 : 16);
-        s.ring_slots = layer_ring_slots(MT);
-        s.ring = take((size_t)(layer_threads(MT) / 32) * s.ring_slots * kSlotBytes);
+        s.ring_slots = layer_ring_slots(MT, nd);
+        s.ring = take((size_t)(layer_threads(MT) / 32) * s.ring_slots * slot_bytes(layer_rows(MT, nd)));
         off = o;
     }
     s.y_off = off;
@@ -838,6 +861,10 @@ __device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, i
 // vectors and the multiply-adds not.
 __device__ __forceinline__ int pair_cost(int K, int m) { return max(1, (K + K / 8) / 256) * (3 + m); }
 
+// The same for an item of RW rows (RW / 2 row pairs).
+template <int RW>
+__device__ __forceinline__ int item_cost(int K, int m) { return pair_cost(K, m) * (RW / 2); }
+
 // The layer, T <= 64 tokens.  MT = tokens per group (vectors per item);
 // kOutRows: one token, down and combine by output rows; kI8: the
 // integer-activation variant (int8 activations, one digit plane).
@@ -848,25 +875,28 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     constexpr int kLayerThreads = layer_threads(MT);
     constexpr int kLayerWarps = kLayerThreads / 32;
     extern __shared__ __align__(16) unsigned char lsm[];
-    constexpr int P_GU = layer_ring_slots(MT);  // ring slots (steps in flight + 1) of the streams
-    constexpr int P_DN = layer_ring_slots(MT);
+    // digits per staged activation: fp32 activations three (21-bit), bf16 two (14-bit), the int8 variant one
+    constexpr int nd = kI8 ? 1 : kBf16 ? 2 : 3;
+    // rows per step of the several-token streams (item = kRW rows: kHP gate/up row pairs, or kRW down rows);
+    // the one-token streams take two
+    constexpr int kRW = layer_rows(MT, nd), kHP = kRW / 2;
+    constexpr int P_GU = layer_ring_slots(MT, nd);  // ring slots (steps in flight + 1) of the streams
+    constexpr int P_DN = P_GU;
     const int H = a.H, F = a.F, E = a.E, k = a.k, T = a.T;
     const int P = T * k;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
-    // digit planes per staged vector: fp32 activations three (21-bit), bf16 two (14-bit), the int8 variant one
-    constexpr int nd = kI8 ? 1 : kBf16 ? 2 : 3;
     constexpr int kPieceChunks = MT == 1 ? 2 : 1;  // router chunks per lane per piece
     // staged vectors as digit planes (16-byte units per vector)
-    const int xvs = digit_vec_units(H);
-    const int hvs = digit_vec_units(F);
+    const int xvs = digit_vec_units(H, nd);
+    const int hvs = digit_vec_units(F, nd);
     unsigned char* xcorr = lsm + ls.x_off + (size_t)ls.nx * xvs * 16;
     float4* hs = reinterpret_cast<float4*>(lsm + ls.h_off);
     unsigned char* hcorr = lsm + ls.h_off + (size_t)ls.nh * hvs * 16;
     const UnionSmem u = union_smem(lsm, ls);
     float* ypart = reinterpret_cast<float*>(lsm + ls.y_off);
-    unsigned char* ring = lsm + ls.ring + (size_t)(threadIdx.x >> 5) * P_GU * kSlotBytes;  // this warp's ring
+    unsigned char* ring = lsm + ls.ring + (size_t)(threadIdx.x >> 5) * P_GU * slot_bytes(kRW);  // this warp's ring
 
     unsigned int* bar_word = launch_barrier_word();
     if (!bar_word) {  // not a cooperative launch: nothing can be synchronised (same answer in every CTA)
@@ -900,18 +930,69 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         stage_vecs(a.h, 0, F, n, row0, nullptr, 1, hs, hcorr, (int)threadIdx.x, kLayerThreads);
     };
 
-    // gate/up item finisher: h[pos_t, n] = silu(gate) * up for the group's vectors
-    auto gateup_finish = [&](int n, int pos0, bool, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+    // Sums of an item's rows over the warp, for each of its vectors: out(r, t, value) runs on one
+    // lane per row r and vector t.  tot is float[RW][MT] (RW = 2 or 4 rows).
+    auto rows_out = [&](const VecSet<MT>& v, const auto& tot, auto out) {
+        constexpr int RW = sizeof(tot) / sizeof(tot[0]);
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
             if (t < v.m) {
-                const float gu = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: gate, lane 16: up
-                const float gv = gu;
-                const float uv = __shfl_sync(0xFFFFFFFFu, gu, 16);
+                if constexpr (RW == 2) {
+                    const float y = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: row 0, lane 16: row 1
+                    if ((lane & 15) == 0) out(lane >> 4, t, y);
+                } else {
+                    const float y = warp_sum4(tot[0][t], tot[1][t], tot[2][t], tot[3][t]);  // row r on lane 8 r
+                    if ((lane & 7) == 0) out(lane >> 3, t, y);
+                }
+            }
+        }
+    };
+    // gate/up item finisher: the item's rows are (gate n0, up n0, gate n0 + 1, up n0 + 1, ...);
+    // h[pos0 + t, n] = silu(gate) * up for the group's vectors
+    auto gateup_finish = [&](int n0, int pos0, const VecSet<MT>& v, const auto& tot) {
+        constexpr int RW = sizeof(tot) / sizeof(tot[0]);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            if (t < v.m) {
+                float gv, uv;
+                int n;
+                bool mine;
+                if constexpr (RW == 2) {
+                    gv = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: gate, lane 16: up
+                    uv = __shfl_sync(0xFFFFFFFFu, gv, 16);
+                    n = n0;
+                    mine = lane == 0;
+                } else {
+                    gv = warp_sum4(tot[0][t], tot[1][t], tot[2][t], tot[3][t]);  // gate/up of n0 on lanes 0/8, of n0 + 1 on 16/24
+                    uv = __shfl_down_sync(0xFFFFFFFFu, gv, 8);
+                    n = n0 + (lane >> 4);
+                    mine = (lane & 15) == 0;
+                }
                 const int pos = pos0 + t;
-                if (lane == 0 && COLI_IN_BOUNDS(pos >= 0 && pos < P + T && n >= 0 && n < F, a.err))
+                if (mine && COLI_IN_BOUNDS(pos >= 0 && pos < P + T && n >= 0 && n < F, a.err))
                     a.h[(size_t)pos * F + n] = gv / (1.0f + expf(-gv)) * uv;
             }
+        }
+    };
+    // an item's rows: gate/up rows row0 .. row0 + RW / 2 - 1 of the stacked [E + 1, F] rows, as
+    // (gate, up) pairs; down rows row0 .. row0 + RW - 1 of the stacked [E + 1, H] rows
+    auto gateup_rows = [&](auto& r, size_t row0) {
+        constexpr int RW = sizeof(r.q) / sizeof(r.q[0]);
+#pragma unroll
+        for (int p = 0; p < RW / 2; ++p) {
+            const size_t row = row0 + p;
+            r.q[2 * p] = a.gate_q + row * (H / 2);
+            r.q[2 * p + 1] = a.up_q + row * (H / 2);
+            r.s[2 * p] = a.gate_s + row * (H / kGroup);
+            r.s[2 * p + 1] = a.up_s + row * (H / kGroup);
+        }
+    };
+    auto down_rows = [&](auto& r, size_t row0) {
+        constexpr int RW = sizeof(r.q) / sizeof(r.q[0]);
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+            r.q[i] = a.down_q + (row0 + i) * (F / 2);
+            r.s[i] = a.down_s + (row0 + i) * (F / kGroup);
         }
     };
 
@@ -942,18 +1023,18 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
         int lo = 0, hi = 0;
         if (kOutRows) {
-        } else if (nseg == 1) {  // one token group: an even split of the F row pairs
+        } else if (nseg == 1) {  // one token group: an even split of the F / kHP items
             if (threadIdx.x == 0) {
                 u.seg_i[0] = 0;
-                u.seg_i[1] = F;
+                u.seg_i[1] = F / kHP;
             }
             __syncthreads();
-            lo = (int)((long long)F * blockIdx.x / gridDim.x);
-            hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
+            lo = (int)((long long)(F / kHP) * blockIdx.x / gridDim.x);
+            hi = (int)((long long)(F / kHP) * (blockIdx.x + 1) / gridDim.x);
         } else {
             for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
-                u.seg_i[s] = F;
-                u.seg_cost[s] = pair_cost(H, min(MT, T - s * MT));
+                u.seg_i[s] = F / kHP;
+                u.seg_cost[s] = item_cost<kRW>(H, min(MT, T - s * MT));
             }
             __syncthreads();
             st = seg_prepare(u, nseg);
@@ -966,13 +1047,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             if (s_lo >= s_hi) continue;
             const int t0 = s * MT, m = min(MT, T - t0);
             const int base = st.ipre[s];
-            auto rows_of = [&](int j, RowPair& r) {
-                const size_t row = (size_t)E * F + (j - base);
-                r.q0 = a.gate_q + row * (H / 2);
-                r.q1 = a.up_q + row * (H / 2);
-                r.s0 = a.gate_s + row * (H / kGroup);
-                r.s1 = a.up_s + row * (H / kGroup);
-            };
+            auto rows_of = [&](int j, Rows<kRW>& r) { gateup_rows(r, (size_t)E * F + kHP * (j - base)); };
             auto vecs_of = [&](int, VecSet<MT>& v) {
                 v.m = m;
 #pragma unroll
@@ -981,8 +1056,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     v.vi[t] = vi;
                 }
             };
-            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
-                gateup_finish(j - base, P + t0, true, v, tot);
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
+                gateup_finish(kHP * (j - base), P + t0, v, tot);
             };
             auto hook = [&]() {
                 if (all_x) {
@@ -995,8 +1070,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of,
-                                       fin, hook);
+            stream_rows<MT, kRW, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
+                                           fin, hook);
             ran = true;
         }
         if constexpr (kOutRows) {
@@ -1097,23 +1172,17 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         {
             const int s_lo = (int)((long long)F * blockIdx.x / gridDim.x);
             const int s_hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
-            auto rows_of = [&](int j, RowPair& r) {
-                const size_t row = (size_t)E * F + j;
-                r.q0 = a.gate_q + row * (H / 2);
-                r.q1 = a.up_q + row * (H / 2);
-                r.s0 = a.gate_s + row * (H / kGroup);
-                r.s1 = a.up_s + row * (H / kGroup);
-            };
+            auto rows_of = [&](int j, Rows<2>& r) { gateup_rows(r, (size_t)E * F + j); };
             auto vecs_of = [&](int, VecSet<MT>& v) {
                 v.m = 1;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) v.vi[t] = 0;
             };
-            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) { gateup_finish(j, P, true, v, tot); };
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) { gateup_finish(j, P, v, tot); };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of,
-                                       fin, route_hook);
+            stream_rows<MT, 2, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
+                                         fin, route_hook);
         }
         stamp(a, 14);
         stamp(a, 4);
@@ -1123,15 +1192,11 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int lo = (int)((long long)total * blockIdx.x / gridDim.x);
         const int hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
         const FastDiv div_f(F, total);
-        auto rows_of = [&](int j, RowPair& r) {
+        auto rows_of = [&](int j, Rows<2>& r) {
             const int g = div_f(j);
             int e = u.gexp[g];
             if (!COLI_IN_BOUNDS(e >= 0 && e < E, a.err)) e = 0;
-            const size_t row = (size_t)e * F + (j - g * F);
-            r.q0 = a.gate_q + row * (H / 2);
-            r.q1 = a.up_q + row * (H / 2);
-            r.s0 = a.gate_s + row * (H / kGroup);
-            r.s1 = a.up_s + row * (H / kGroup);
+            gateup_rows(r, (size_t)e * F + (j - g * F));
         };
         auto vecs_of = [&](int, VecSet<MT>& v) {
             v.m = 1;
@@ -1142,11 +1207,11 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         };
         auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
             const int g = div_f(j);
-            gateup_finish(j - g * F, g, false, v, tot);
+            gateup_finish(j - g * F, g, v, tot);
         };
         const int first = lo + warp;
         const int nj = first < hi ? (hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-        stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of, fin);
+        stream_rows<MT, 2, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of, fin);
     } else {
         const bool scored_here = all_x;  // the kernel scored the tokens (pieces summed into shared memory)
         if (scored_here) sum_pieces();
@@ -1221,13 +1286,13 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
             if (s < n_sd) {
                 const int m = min(MT, T - s * MT);
-                u.seg_i[s] = H / 2;
-                u.seg_cost[s] = pair_cost(F, m);
+                u.seg_i[s] = H / kRW;
+                u.seg_cost[s] = item_cost<kRW>(F, m);
             } else {
                 const int g = s - n_sd, e = u.gexp[g];
                 const int m = min(MT, u.off[e] + u.cnt[e] - u.gpos[g]);
-                u.seg_i[s] = F;
-                u.seg_cost[s] = pair_cost(H, m);
+                u.seg_i[s] = F / kHP;
+                u.seg_cost[s] = item_cost<kRW>(H, m);
             }
         }
         __syncthreads();
@@ -1245,13 +1310,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             stage_h(m, P + t0);
             __syncthreads();
             const int base = st.ipre[s];
-            auto rows_of = [&](int j, RowPair& r) {
-                const size_t row = (size_t)E * H + 2 * (j - base);
-                r.q0 = a.down_q + row * (F / 2);
-                r.q1 = r.q0 + F / 2;
-                r.s0 = a.down_s + row * (F / kGroup);
-                r.s1 = r.s0 + F / kGroup;
-            };
+            auto rows_of = [&](int j, Rows<kRW>& r) { down_rows(r, (size_t)E * H + kRW * (j - base)); };
             auto vecs_of = [&](int, VecSet<MT>& v) {
                 v.m = m;
 #pragma unroll
@@ -1259,19 +1318,16 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     v.vi[t] = t;
                 }
             };
-            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
-                const int n = 2 * (j - base);
-#pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    if (t < v.m) {
-                        const float y = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: row n, lane 16: row n + 1
-                        if ((lane & 15) == 0) a.y[(size_t)(P + t0 + t) * H + n + (lane >> 4)] = y;
-                    }
-                }
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
+                const int n0 = kRW * (j - base);
+                rows_out(v, tot, [&](int r, int t, float y) {
+                    if (COLI_IN_BOUNDS(n0 + r < H, a.err)) a.y[(size_t)(P + t0 + t) * H + n0 + r] = y;
+                });
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin);
+            stream_rows<MT, kRW, P_DN, nd>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of,
+                                           fin);
         }
 
         stamp(a, 14);
@@ -1295,15 +1351,11 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 __syncthreads();
             }
             auto seg_of = [&](int j) { return all_x ? last_le(st.ipre, nseg - 1, j) : s; };
-            auto rows_of = [&](int j, RowPair& r) {
+            auto rows_of = [&](int j, Rows<kRW>& r) {
                 const int sj = seg_of(j);
                 int e = u.gexp[sj - n_sd];
-                if (!COLI_IN_BOUNDS(e >= 0 && e < E && j - st.ipre[sj] < F, a.err)) e = 0;
-                const size_t row = (size_t)e * F + (j - st.ipre[sj]);
-                r.q0 = a.gate_q + row * (H / 2);
-                r.q1 = a.up_q + row * (H / 2);
-                r.s0 = a.gate_s + row * (H / kGroup);
-                r.s1 = a.up_s + row * (H / kGroup);
+                if (!COLI_IN_BOUNDS(e >= 0 && e < E && j - st.ipre[sj] < F / kHP, a.err)) e = 0;
+                gateup_rows(r, (size_t)e * F + kHP * (j - st.ipre[sj]));
             };
             auto vecs_of = [&](int j, VecSet<MT>& v) {
                 const int g = seg_of(j) - n_sd, e = u.gexp[g], p0 = u.gpos[g];
@@ -1314,13 +1366,14 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     v.vi[t] = vi;
                 }
             };
-            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
                 const int sj = seg_of(j);
-                gateup_finish(j - st.ipre[sj], u.gpos[sj - n_sd], false, v, tot);
+                gateup_finish(kHP * (j - st.ipre[sj]), u.gpos[sj - n_sd], v, tot);
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_GU>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, nd, ring, rows_of, vecs_of, fin);
+            stream_rows<MT, kRW, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
+                                           fin);
         }
     }
     stamp(a, 5);
@@ -1340,15 +1393,11 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
         const int n_slots = n_kept + 1;
         const FastDiv div_pr(npr, (long long)npr * n_slots);
-        auto rows_of = [&](int j, RowPair& r) {
+        auto rows_of = [&](int j, Rows<2>& r) {
             const int slot = div_pr(j), pr = pr_lo + (j - slot * npr);
             int e = slot < n_kept ? u.gexp[slot] : E;
             if (!COLI_IN_BOUNDS(e >= 0 && e <= E && 2 * pr + 1 < H, a.err)) e = 0;
-            const size_t row = (size_t)e * H + 2 * pr;
-            r.q0 = a.down_q + row * (F / 2);
-            r.q1 = r.q0 + F / 2;
-            r.s0 = a.down_s + row * (F / kGroup);
-            r.s1 = r.s0 + F / kGroup;
+            down_rows(r, (size_t)e * H + 2 * pr);
         };
         auto vecs_of = [&](int j, VecSet<MT>& v) {
             const int slot = div_pr(j);
@@ -1381,8 +1430,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int total = npr * n_slots;
         const int first = warp;
         const int nj = first < total ? (total - first + kLayerWarps - 1) / kLayerWarps : 0;
-        stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin,
-                                   hook);
+        stream_rows<MT, 2, P_DN, nd>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin,
+                                     hook);
         __syncthreads();
         stamp(a, 8);
         for (int i = threadIdx.x; i < 2 * npr; i += kLayerThreads) {
@@ -1401,8 +1450,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
             const int e = u.gexp[s];
             const int m = min(MT, u.off[e] + u.cnt[e] - u.gpos[s]);
-            u.seg_i[s] = H / 2;
-            u.seg_cost[s] = pair_cost(F, m);
+            u.seg_i[s] = H / kRW;
+            u.seg_cost[s] = item_cost<kRW>(F, m);
         }
         __syncthreads();
         const SegTable st = seg_prepare(u, nseg);
@@ -1417,13 +1466,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             stage_h(m, p0);
             __syncthreads();
             const int base = st.ipre[s];
-            auto rows_of = [&](int j, RowPair& r) {
-                const size_t row = (size_t)e * H + 2 * (j - base);
-                r.q0 = a.down_q + row * (F / 2);
-                r.q1 = r.q0 + F / 2;
-                r.s0 = a.down_s + row * (F / kGroup);
-                r.s1 = r.s0 + F / kGroup;
-            };
+            auto rows_of = [&](int j, Rows<kRW>& r) { down_rows(r, (size_t)e * H + kRW * (j - base)); };
             auto vecs_of = [&](int, VecSet<MT>& v) {
                 v.m = m;
 #pragma unroll
@@ -1431,22 +1474,19 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     v.vi[t] = t;
                 }
             };
-            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
-                const int n = 2 * (j - base);
-#pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    if (t < v.m) {
-                        const float y = warp_sum2(tot[0][t], tot[1][t]);  // lane 0: row n, lane 16: row n + 1
-                        if ((lane & 15) == 0 && COLI_IN_BOUNDS(p0 + t < P && n + 1 < H, a.err)) {
-                            const float wt = u.w[u.perm[p0 + t]];
-                            a.y[(size_t)(p0 + t) * H + n + (lane >> 4)] = wt * y;
-                        }
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
+                const int n0 = kRW * (j - base);
+                rows_out(v, tot, [&](int r, int t, float y) {
+                    if (COLI_IN_BOUNDS(p0 + t < P && n0 + r < H, a.err)) {
+                        const float wt = u.w[u.perm[p0 + t]];
+                        a.y[(size_t)(p0 + t) * H + n0 + r] = wt * y;
                     }
-                }
+                });
             };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_row_pairs<MT, P_DN>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, nd, ring, rows_of, vecs_of, fin);
+            stream_rows<MT, kRW, P_DN, nd>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of,
+                                           fin);
         }
         stamp(a, 7);
         grid_barrier(bar, deadline, a.err);
