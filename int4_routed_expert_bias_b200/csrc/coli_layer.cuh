@@ -38,6 +38,7 @@
 #pragma once
 
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "coli_int4.cuh"
 #include "coli_router.cuh"
@@ -459,45 +460,6 @@ __host__ __device__ inline LayerSmem layer_smem(int T, int H, int F, int E, int 
 // ---------------------------------------------------------------------------
 // small block-level helpers (every thread of the block calls them)
 
-// Exclusive prefix sum of v[0..n) in place (int), returns the total.
-__device__ __forceinline__ int block_excl_scan(int* v, int n, int* tmp32)
-{
-    // each thread owns a contiguous run
-    const int nthr = blockDim.x, nwarp = nthr >> 5;
-    const int per = (n + nthr - 1) / nthr;
-    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
-    int s = 0;
-    for (int i = lo; i < hi; ++i) s += v[i];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) tmp32[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nwarp ? tmp32[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
-            if (lane >= o) w += y;
-        }
-        if (lane < nwarp) tmp32[lane] = w;  // inclusive warp totals
-    }
-    __syncthreads();
-    int run = incl - s + (warp > 0 ? tmp32[warp - 1] : 0);
-    const int total = tmp32[nwarp - 1];
-    for (int i = lo; i < hi; ++i) {
-        const int x = v[i];
-        v[i] = run;
-        run += x;
-    }
-    __syncthreads();
-    return total;
-}
-
 // Segment lookup: the segment s with pre[s] <= x < pre[s + 1] (pre ascending, pre[0] = 0).
 __device__ __forceinline__ int seg_find(const int* pre, int nseg, long long x)
 {
@@ -662,46 +624,8 @@ __device__ __noinline__ void topk_rounds_global(const float* __restrict__ part, 
 // ---------------------------------------------------------------------------
 // the kernel
 
-// 64-bit exclusive prefix sum of v[0..n) in place; returns the total.
-__device__ __forceinline__ long long block_excl_scan64(long long* v, int n, long long* tmp32)
-{
-    const int nthr = blockDim.x, nwarp = nthr >> 5;
-    const int per = (n + nthr - 1) / nthr;
-    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
-    long long s = 0;
-    for (int i = lo; i < hi; ++i) s += v[i];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    long long incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const long long y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) tmp32[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        long long w = lane < nwarp ? tmp32[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const long long y = __shfl_up_sync(0xFFFFFFFFu, w, o);
-            if (lane >= o) w += y;
-        }
-        if (lane < nwarp) tmp32[lane] = w;
-    }
-    __syncthreads();
-    long long run = incl - s + (warp > 0 ? tmp32[warp - 1] : 0);
-    const long long total = tmp32[nwarp - 1];
-    for (int i = lo; i < hi; ++i) {
-        const long long x = v[i];
-        v[i] = run;
-        run += x;
-    }
-    __syncthreads();
-    return total;
-}
-
 // Work-list segments of one phase: segment s holds n items of cost c each.
-// After seg_prepare, ipre[s] / cpre[s] are the item / cost offsets of segment s
+// Once built (seg_build_warp), ipre[s] / cpre[s] are the item / cost offsets of segment s
 // (ipre[nseg], cpre[nseg] the totals).
 struct SegTable {
     int* ipre;        // [nseg + 1]
@@ -780,20 +704,116 @@ __device__ __forceinline__ UnionSmem union_smem(unsigned char* base, const Layer
 }
 
 
-// Prefix sums of a segment table whose counts are in ipre[0..n) and per-item
-// costs in cost[0..n) (all threads call this).
-__device__ __forceinline__ SegTable seg_prepare(const UnionSmem& u, int nseg)
+// A segment table built by one warp: segment s < nseg has items_of(s) items
+// of cost_of(s) each; ipre / cpre get the item / cost offsets of s = 0..nseg
+// (exclusive prefix sums, the totals at nseg) and cost the per-item costs.
+// Each lane takes a contiguous run of segments; two warp scans join them.  The
+// caller synchronises the block before the table is read.
+template <typename ItemsOf, typename CostOf>
+__device__ __forceinline__ void seg_build_warp(const UnionSmem& u, int nseg, ItemsOf items_of, CostOf cost_of)
 {
-    SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
-    for (int s = threadIdx.x; s < nseg; s += blockDim.x) st.cpre[s] = (long long)st.ipre[s] * st.cost[s];
-    if (threadIdx.x == 0) {
-        st.ipre[nseg] = 0;
-        st.cpre[nseg] = 0;
+    const int lane = threadIdx.x & 31;
+    const int per = (nseg + 1 + 31) / 32;
+    const int s_lo = min(nseg + 1, lane * per), s_hi = min(nseg + 1, s_lo + per);
+    int isum = 0;
+    long long csum = 0;
+    for (int s = s_lo; s < s_hi && s < nseg; ++s) {
+        const int n = items_of(s);
+        isum += n;
+        csum += (long long)n * cost_of(s);
     }
-    __syncthreads();
-    block_excl_scan(st.ipre, nseg + 1, reinterpret_cast<int*>(u.tmp));
-    block_excl_scan64(st.cpre, nseg + 1, u.tmp);
-    return st;
+    int iinc = isum;
+    long long cinc = csum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, iinc, o);
+        const long long yc = __shfl_up_sync(0xFFFFFFFFu, cinc, o);
+        if (lane >= o) {
+            iinc += y;
+            cinc += yc;
+        }
+    }
+    int ip = iinc - isum;
+    long long cp = cinc - csum;
+    for (int s = s_lo; s < s_hi; ++s) {
+        u.seg_i[s] = ip;
+        u.seg_c[s] = cp;
+        if (s < nseg) {
+            const int n = items_of(s), c = cost_of(s);
+            u.seg_cost[s] = c;
+            ip += n;
+            cp += (long long)n * c;
+        }
+    }
+}
+
+// The batch union by one warp (T <= 64 tokens, their k slots in idx, dropped
+// slots -1): per expert the token mask, count, first sorted position (off) and
+// first group (gpre, groups of up to MT pairs), the sorted pair list perm and
+// each pair's position ipos (experts ascending, pairs ascending within an
+// expert), and per group its expert and first position.  Each lane takes a
+// contiguous run of experts; warp scans give the offsets.  Returns the number
+// of groups (also at gpre[E]).  The caller synchronises the block afterwards.
+template <int MT>
+__device__ __forceinline__ int union_warp(const UnionSmem& u, int T, int k, int E, int* err)
+{
+    const int lane = threadIdx.x & 31;
+    const int P = T * k;
+    for (int e = lane; e < E; e += 32) u.mask[e] = 0ull;
+    __syncwarp();
+    for (int p = lane; p < P; p += 32) {
+        const int e = u.idx[p];
+        if (e >= 0 && COLI_IN_BOUNDS(e < E, err)) atomicOr(&u.mask[e], 1ull << (p / k));  // dropped slots: none
+    }
+    __syncwarp();
+    const int per = (E + 31) / 32;
+    const int e_lo = min(E, lane * per), e_hi = min(E, e_lo + per);
+    int cs = 0, gs = 0;
+    for (int e = e_lo; e < e_hi; ++e) {
+        const int c = __popcll(u.mask[e]);
+        cs += c;
+        gs += (c + MT - 1) / MT;
+    }
+    int ci = cs, gi = gs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, ci, o);
+        const int yg = __shfl_up_sync(0xFFFFFFFFu, gi, o);
+        if (lane >= o) {
+            ci += y;
+            gi += yg;
+        }
+    }
+    const int n_pairs = __shfl_sync(0xFFFFFFFFu, ci, 31), n_groups = __shfl_sync(0xFFFFFFFFu, gi, 31);
+    int oc = ci - cs, og = gi - gs;
+    for (int e = e_lo; e < e_hi; ++e) {
+        const int c = __popcll(u.mask[e]);
+        u.cnt[e] = c;
+        u.off[e] = oc;
+        u.gpre[e] = og;
+        for (int i = 0; i * MT < c; ++i, ++og) {
+            u.gexp[og] = e;
+            u.gpos[og] = oc + i * MT;
+        }
+        oc += c;
+    }
+    if (lane == 0) {
+        u.off[E] = n_pairs;
+        u.gpre[E] = n_groups;
+    }
+    __syncwarp();
+    for (int p = lane; p < P; p += 32) {
+        const int t = p / k, e = u.idx[p];
+        int pos = -1;
+        if (e >= 0 && e < E) {
+            const unsigned long long below = t == 0 ? 0ull : (u.mask[e] & ((1ull << t) - 1ull));
+            pos = u.off[e] + __popcll(below);
+            if (COLI_IN_BOUNDS(pos < P, err)) u.perm[pos] = p;
+            else pos = -1;
+        }
+        u.ipos[p] = pos;
+    }
+    return n_groups;
 }
 
 }  // namespace coli
@@ -856,14 +876,16 @@ __device__ __forceinline__ void router_piece(const LayerArgs& a, int e, int p, i
     }
 }
 
-// Cost per item of a row-pair item of m vectors: bytes of the two rows (in
-// 256-byte units) times (3 + m) / 4, the int4 decode being shared by the
-// vectors and the multiply-adds not.
-__device__ __forceinline__ int pair_cost(int K, int m) { return max(1, (K + K / 8) / 256) * (3 + m); }
-
-// The same for an item of RW rows (RW / 2 row pairs).
-template <int RW>
-__device__ __forceinline__ int item_cost(int K, int m) { return pair_cost(K, m) * (RW / 2); }
+// Cost of an item of RW rows (RW / 2 row pairs) against m vectors of ND
+// digits: bytes of the rows (in 256-byte units) times (c + m), the int4 decode
+// and the copies being shared by the vectors and the multiply-adds not; c, the
+// per-byte share, measured best at 2 for two-digit vectors (four rows a step)
+// and 3 otherwise.
+template <int RW, int ND>
+__device__ __forceinline__ int item_cost(int K, int m)
+{
+    return max(1, (K + K / 8) / 256) * ((ND == 2 ? 2 : 3) + m) * (RW / 2);
+}
 
 // The layer, T <= 64 tokens.  MT = tokens per group (vectors per item);
 // kOutRows: one token, down and combine by output rows; kI8: the
@@ -996,6 +1018,11 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         }
     };
 
+    // The CTA's items j = lo, lo + 1, ... go to its warps round-robin, continued across segments: the
+    // first item of a segment that starts d items into the CTA's range belongs to warp d mod warps,
+    // and this warp's first item of the segment is deal(d) items into it.
+    auto deal = [&](int d) { return ((warp - d) % kLayerWarps + kLayerWarps) % kLayerWarps; };
+
     // ======================= phase A: router pieces, shared gate/up =======================
     {
         // Router pieces (scored here up to 4 tokens): block b takes pieces b, b + G, ... and its
@@ -1023,21 +1050,21 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
         int lo = 0, hi = 0;
         if (kOutRows) {
-        } else if (nseg == 1) {  // one token group: an even split of the F / kHP items
+        } else if (nseg == 1) {
+            // one token group: an even split of the F row pairs, streamed two rows a step through a ring
+            // of twice the slots (a warp holds about one item: its steps are then nearly all in flight)
             if (threadIdx.x == 0) {
                 u.seg_i[0] = 0;
-                u.seg_i[1] = F / kHP;
+                u.seg_i[1] = F;
             }
             __syncthreads();
-            lo = (int)((long long)(F / kHP) * blockIdx.x / gridDim.x);
-            hi = (int)((long long)(F / kHP) * (blockIdx.x + 1) / gridDim.x);
+            lo = (int)((long long)F * blockIdx.x / gridDim.x);
+            hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
         } else {
-            for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
-                u.seg_i[s] = F / kHP;
-                u.seg_cost[s] = item_cost<kRW>(H, min(MT, T - s * MT));
-            }
+            if (warp == 0)
+                seg_build_warp(
+                    u, nseg, [&](int) { return F / kHP; }, [&](int s) { return item_cost<kRW, nd>(H, min(MT, T - s * MT)); });
             __syncthreads();
-            st = seg_prepare(u, nseg);
             seg_cta_range(st, lo, hi);
         }
         stamp(a, 10);
@@ -1047,33 +1074,39 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             if (s_lo >= s_hi) continue;
             const int t0 = s * MT, m = min(MT, T - t0);
             const int base = st.ipre[s];
-            auto rows_of = [&](int j, Rows<kRW>& r) { gateup_rows(r, (size_t)E * F + kHP * (j - base)); };
-            auto vecs_of = [&](int, VecSet<MT>& v) {
-                v.m = m;
+            auto run = [&](auto rows_c) {  // rows per step RW (items of RW / 2 row pairs)
+                constexpr int RW = decltype(rows_c)::value, HP = RW / 2, R = P_GU * kRW / RW;
+                auto rows_of = [&](int j, Rows<RW>& r) { gateup_rows(r, (size_t)E * F + HP * (j - base)); };
+                auto vecs_of = [&](int, VecSet<MT>& v) {
+                    v.m = m;
 #pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    const int vi = all_x ? t0 + t : t;
-                    v.vi[t] = vi;
-                }
+                    for (int t = 0; t < MT; ++t) {
+                        const int vi = all_x ? t0 + t : t;
+                        v.vi[t] = vi;
+                    }
+                };
+                auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[RW][MT]) {
+                    gateup_finish(HP * (j - base), P + t0, v, tot);
+                };
+                auto hook = [&]() {
+                    if (all_x) {
+                        if (!ran) stage_all();
+                    } else {  // this group's tokens (the router ran before the launch)
+                        __syncthreads();
+                        stage_x(m, t0);
+                        __syncthreads();
+                    }
+                };
+                const int first = s_lo + deal(s_lo - lo);
+                const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
+                stream_rows<MT, RW, R, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of,
+                                           vecs_of, fin, hook);
             };
-            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
-                gateup_finish(kHP * (j - base), P + t0, v, tot);
-            };
-            auto hook = [&]() {
-                if (all_x) {
-                    if (!ran) stage_all();
-                } else {  // this group's tokens (the router ran before the launch)
-                    __syncthreads();
-                    stage_x(m, t0);
-                    __syncthreads();
-                }
-            };
-            const int first = s_lo + warp;
-            const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_rows<MT, kRW, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
-                                           fin, hook);
+            if (nseg == 1) run(std::integral_constant<int, 2>{});
+            else run(std::integral_constant<int, kRW>{});
             ran = true;
         }
+        stamp(a, 15);
         if constexpr (kOutRows) {
             // one token, nothing streams in this phase: the router pieces (their weight loads the longest
             // latency here) run on the last rw warps beside the staging of x on the others
@@ -1102,19 +1135,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int S1 = k + 1;  // one token: slots (routed in order, shared last)
     const int pr_lo = (int)((long long)(H / 2) * blockIdx.x / gridDim.x);  // one token: this CTA's output row pairs
     const int npr = (int)((long long)(H / 2) * (blockIdx.x + 1) / gridDim.x) - pr_lo;
-    float* s_logit = reinterpret_cast<float*>(lsm + ls.logit);
     const int npc = a.n_pieces == 0 ? (gH.per_lane + kPieceChunks - 1) / kPieceChunks : a.n_pieces;
-    // router scores of the tokens: sums of the per-piece partials (independent loads), into shared memory
-    auto sum_pieces = [&]() {
-        for (int i = threadIdx.x; i < T * E; i += kLayerThreads) {
-            float v = 0.f;
-#pragma unroll
-            for (int p = 0; p < 16; ++p)
-                if (p < npc) v += a.logit_part[(size_t)p * T * E + i];
-            s_logit[i] = v;
-        }
-        __syncthreads();
-    };
+    float* s_logit = reinterpret_cast<float*>(lsm + ls.logit);
     if constexpr (kOutRows) {
         // The shared expert's gate/up rows need no routing: this CTA's share of them (an even split)
         // has its first loads issued, then (hook) the token is scored and routed while no warp
@@ -1213,8 +1235,19 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int nj = first < hi ? (hi - first + kLayerWarps - 1) / kLayerWarps : 0;
         stream_rows<MT, 2, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of, fin);
     } else {
-        const bool scored_here = all_x;  // the kernel scored the tokens (pieces summed into shared memory)
-        if (scored_here) sum_pieces();
+        const bool scored_here = all_x;  // the kernel scored the tokens (npc partial pieces per score)
+        if (scored_here) {
+            // the scores: sums of the pieces (independent loads, every thread), into shared memory
+            for (int i = threadIdx.x; i < T * E; i += kLayerThreads) {
+                float v = 0.f;
+#pragma unroll
+                for (int p = 0; p < 16; ++p)
+                    if (p < npc) v += a.logit_part[(size_t)p * T * E + i];
+                s_logit[i] = v;
+            }
+            __syncthreads();
+        }
+        // top-k: one warp per token
         for (int t = warp; t < T; t += kLayerWarps) {
             int my_e;
             float my_w;
@@ -1239,64 +1272,25 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             }
         }
         stamp(a, 11);
-        for (int e = threadIdx.x; e < E; e += kLayerThreads) u.mask[e] = 0ull;
         __syncthreads();
-        // union: token masks per expert, counts, offsets, stable positions
-        for (int p = threadIdx.x; p < P; p += kLayerThreads)
-            if (u.idx[p] >= 0 && COLI_IN_BOUNDS(u.idx[p] < E, a.err))  // dropped slots (-1) have no expert
-                atomicOr(&u.mask[u.idx[p]], 1ull << (p / k));
-        __syncthreads();
-        for (int e = threadIdx.x; e <= E; e += kLayerThreads) {
-            const int c = e < E ? __popcll(u.mask[e]) : 0;
-            u.off[e] = c;
-            u.gpre[e] = (c + MT - 1) / MT;
-            if (e < E) u.cnt[e] = c;
-        }
-        __syncthreads();
-        block_excl_scan(u.off, E + 1, reinterpret_cast<int*>(u.tmp));
-        const int n_rg = block_excl_scan(u.gpre, E + 1, reinterpret_cast<int*>(u.tmp));
-        for (int p = threadIdx.x; p < P; p += kLayerThreads) {
-            const int t = p / k, e = u.idx[p];
-            if (e < 0) {
-                u.ipos[p] = -1;
-                continue;
-            }
-            const unsigned long long below = t == 0 ? 0ull : (u.mask[e] & ((1ull << t) - 1ull));
-            const int pos = u.off[e] + __popcll(below);
-            if (!COLI_IN_BOUNDS(e < E && pos < P, a.err)) {
-                u.ipos[p] = -1;
-                continue;
-            }
-            u.perm[pos] = p;
-            u.ipos[p] = pos;
-        }
-        for (int e = threadIdx.x; e < E; e += kLayerThreads) {
-            const int c = u.cnt[e];
-            for (int i = 0, g = u.gpre[e]; i * MT < c; ++i, ++g) {
-                u.gexp[g] = e;
-                u.gpos[g] = u.off[e] + i * MT;
-            }
-        }
-        __syncthreads();
-
-        stamp(a, 12);
-        // segments: [shared down groups (several tokens)] + routed gate/up groups
+        // union and the segment table of this phase by warp 0:
+        // [shared down groups (several tokens)] + routed gate/up groups
         const int n_sd = kOutRows ? 0 : n_sg;
-        const int nseg = n_sd + n_rg;
-        for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
-            if (s < n_sd) {
-                const int m = min(MT, T - s * MT);
-                u.seg_i[s] = H / kRW;
-                u.seg_cost[s] = item_cost<kRW>(F, m);
-            } else {
-                const int g = s - n_sd, e = u.gexp[g];
-                const int m = min(MT, u.off[e] + u.cnt[e] - u.gpos[g]);
-                u.seg_i[s] = F / kHP;
-                u.seg_cost[s] = item_cost<kRW>(H, m);
-            }
+        if (warp == 0) {
+            const int n_rg = union_warp<MT>(u, T, k, E, a.err);
+            __syncwarp();
+            seg_build_warp(
+                u, n_sd + n_rg, [&](int s) { return s < n_sd ? H / kRW : F / kHP; },
+                [&](int s) {
+                    if (s < n_sd) return item_cost<kRW, nd>(F, min(MT, T - s * MT));
+                    const int g = s - n_sd, e = u.gexp[g];
+                    return item_cost<kRW, nd>(H, min(MT, u.off[e] + u.cnt[e] - u.gpos[g]));
+                });
         }
         __syncthreads();
-        const SegTable st = seg_prepare(u, nseg);
+        stamp(a, 12);
+        const int nseg = n_sd + u.gpre[E];
+        const SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
         int lo, hi;
         seg_cta_range(st, lo, hi);
 
@@ -1324,7 +1318,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     if (COLI_IN_BOUNDS(n0 + r < H, a.err)) a.y[(size_t)(P + t0 + t) * H + n0 + r] = y;
                 });
             };
-            const int first = s_lo + warp;
+            const int first = s_lo + deal(s_lo - lo);
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
             stream_rows<MT, kRW, P_DN, nd>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of,
                                            fin);
@@ -1370,7 +1364,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 const int sj = seg_of(j);
                 gateup_finish(kHP * (j - st.ipre[sj]), u.gpos[sj - n_sd], v, tot);
             };
-            const int first = s_lo + warp;
+            const int first = s_lo + deal(s_lo - lo);
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
             stream_rows<MT, kRW, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
                                            fin);
@@ -1445,16 +1439,16 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         }
     } else {
         // several tokens: routed down rows, one partial output row per pair (routing weight applied)
-        const int n_rg = u.gpre[E];
-        const int nseg = n_rg;
-        for (int s = threadIdx.x; s < nseg; s += kLayerThreads) {
-            const int e = u.gexp[s];
-            const int m = min(MT, u.off[e] + u.cnt[e] - u.gpos[s]);
-            u.seg_i[s] = H / kRW;
-            u.seg_cost[s] = item_cost<kRW>(F, m);
-        }
+        const int nseg = u.gpre[E];  // routed groups
+        if (warp == 0)
+            seg_build_warp(
+                u, nseg, [&](int) { return H / kRW; },
+                [&](int s) {
+                    const int e = u.gexp[s];
+                    return item_cost<kRW, nd>(F, min(MT, u.off[e] + u.cnt[e] - u.gpos[s]));
+                });
         __syncthreads();
-        const SegTable st = seg_prepare(u, nseg);
+        const SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
         int lo, hi;
         seg_cta_range(st, lo, hi);
         for (int s = 0; s < nseg; ++s) {
@@ -1483,7 +1477,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     }
                 });
             };
-            const int first = s_lo + warp;
+            const int first = s_lo + deal(s_lo - lo);
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
             stream_rows<MT, kRW, P_DN, nd>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of,
                                            fin);
