@@ -38,7 +38,6 @@
 #pragma once
 
 #include <cooperative_groups.h>
-#include <type_traits>
 
 #include "coli_int4.cuh"
 #include "coli_router.cuh"
@@ -1025,96 +1024,56 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 
     // ======================= phase A: router pieces, shared gate/up =======================
     {
-        // Router pieces (scored here up to 4 tokens): block b takes pieces b, b + G, ... and its
-        // warps one each, so every block has about the same number.  The shared expert's gate/up
-        // rows are cut into equal-cost ranges.  The first gate/up loads are issued before the
-        // activations are staged and before the warp's router piece is computed (engine hook).
+        // Tokens scored here (one token group): the activations are staged and the router pieces
+        // (block b takes pieces b, b + G, ...; about the same number per block) computed side by side;
+        // the shared expert streams in phases B (gate/up, beside the routing) and C (down).
+        // Larger batches (scored before the launch): the shared expert's gate/up rows of every token
+        // group, cut into equal-cost ranges, each group's activations staged in the stream's hook.
         const int nrp = a.n_pieces == 0 ? (gH.per_lane + kPieceChunks - 1) / kPieceChunks : 0;  // pieces per row
-        // The router pieces read the activations from global memory and are needed only after the
-        // grid barrier, so a warp takes its pieces after its gate/up items (their loads overlap the
-        // other warps' streams); the warps are dealt the pieces from the last warp down, since the
-        // first warps hold the gate/up items.
-        auto router_pieces = [&]() {
-            const int total = E * nrp;
-            for (int i = blockIdx.x + gridDim.x * (kLayerWarps - 1 - warp); i < total; i += gridDim.x * kLayerWarps)
-                router_piece<MT, kBf16, kPieceChunks>(a, i / nrp, i % nrp, T, gH);
-        };
-        auto stage_all = [&]() {
-            stage_x(T, 0);
-            __syncthreads();
-            stamp(a, 1);
-        };
-        // one token: the activations and the router only; the shared expert's rows stream in phase B
-        // (their first loads in flight while the token is routed) and C
-        const int nseg = kOutRows ? 0 : n_sg;
-        SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
-        int lo = 0, hi = 0;
-        if (kOutRows) {
-        } else if (nseg == 1) {
-            // one token group: an even split of the F row pairs, streamed two rows a step through a ring
-            // of twice the slots (a warp holds about one item: its steps are then nearly all in flight)
-            if (threadIdx.x == 0) {
-                u.seg_i[0] = 0;
-                u.seg_i[1] = F;
-            }
-            __syncthreads();
-            lo = (int)((long long)F * blockIdx.x / gridDim.x);
-            hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
-        } else {
+        const int nseg = all_x ? 0 : n_sg;
+        if (nseg > 0) {
+            const SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
             if (warp == 0)
                 seg_build_warp(
                     u, nseg, [&](int) { return F / kHP; }, [&](int s) { return item_cost<kRW, nd>(H, min(MT, T - s * MT)); });
             __syncthreads();
+            int lo, hi;
             seg_cta_range(st, lo, hi);
-        }
-        stamp(a, 10);
-        bool ran = false;
-        for (int s = 0; s < nseg; ++s) {
-            const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
-            if (s_lo >= s_hi) continue;
-            const int t0 = s * MT, m = min(MT, T - t0);
-            const int base = st.ipre[s];
-            auto run = [&](auto rows_c) {  // rows per step RW (items of RW / 2 row pairs)
-                constexpr int RW = decltype(rows_c)::value, HP = RW / 2, R = P_GU * kRW / RW;
-                auto rows_of = [&](int j, Rows<RW>& r) { gateup_rows(r, (size_t)E * F + HP * (j - base)); };
+            stamp(a, 10);
+            for (int s = 0; s < nseg; ++s) {
+                const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
+                if (s_lo >= s_hi) continue;
+                const int t0 = s * MT, m = min(MT, T - t0);
+                const int base = st.ipre[s];
+                auto rows_of = [&](int j, Rows<kRW>& r) { gateup_rows(r, (size_t)E * F + kHP * (j - base)); };
                 auto vecs_of = [&](int, VecSet<MT>& v) {
                     v.m = m;
 #pragma unroll
-                    for (int t = 0; t < MT; ++t) {
-                        const int vi = all_x ? t0 + t : t;
-                        v.vi[t] = vi;
-                    }
+                    for (int t = 0; t < MT; ++t) v.vi[t] = t;
                 };
-                auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[RW][MT]) {
-                    gateup_finish(HP * (j - base), P + t0, v, tot);
+                auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
+                    gateup_finish(kHP * (j - base), P + t0, v, tot);
                 };
-                auto hook = [&]() {
-                    if (all_x) {
-                        if (!ran) stage_all();
-                    } else {  // this group's tokens (the router ran before the launch)
-                        __syncthreads();
-                        stage_x(m, t0);
-                        __syncthreads();
-                    }
+                auto hook = [&]() {  // this group's tokens
+                    __syncthreads();
+                    stage_x(m, t0);
+                    __syncthreads();
                 };
                 const int first = s_lo + deal(s_lo - lo);
                 const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-                stream_rows<MT, RW, R, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of,
-                                           vecs_of, fin, hook);
-            };
-            if (nseg == 1) run(std::integral_constant<int, 2>{});
-            else run(std::integral_constant<int, kRW>{});
-            ran = true;
+                stream_rows<MT, kRW, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of,
+                                               vecs_of, fin, hook);
+            }
         }
         stamp(a, 15);
-        if constexpr (kOutRows) {
-            // one token, nothing streams in this phase: the router pieces (their weight loads the longest
-            // latency here) run on the last rw warps beside the staging of x on the others
+        if (all_x) {
+            // nothing streams in this phase: the router pieces (their weight loads the longest latency
+            // here) run on the last rw warps beside the staging of x on the others
             const int per_cta = (E * nrp + (int)gridDim.x - 1) / (int)gridDim.x;
-            const int rw = max(1, min(kLayerWarps - 4, per_cta));
+            const int rw = max(1, min(kLayerWarps - (T > 1 ? 8 : 4), per_cta));
             const int xw = kLayerWarps - rw;
             if (warp < xw) {
-                stage_vecs(a.x, kBf16 ? 1 : 0, H, 1, 0, nullptr, 1, xs, xcorr, (int)threadIdx.x, xw * 32);
+                stage_vecs(a.x, kBf16 ? 1 : 0, H, T, 0, nullptr, 1, xs, xcorr, (int)threadIdx.x, xw * 32);
             } else {
                 const int total = E * nrp;
                 for (int i = blockIdx.x + gridDim.x * (warp - xw); i < total; i += gridDim.x * rw)
@@ -1122,9 +1081,6 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             }
             __syncthreads();
             stamp(a, 1);
-        } else {
-            if (!ran && all_x) stage_all();  // no gate/up rows in this block: the activations only
-            if (all_x) router_pieces();
         }
     }
     stamp(a, 2);
@@ -1274,8 +1230,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         stamp(a, 11);
         __syncthreads();
         // union and the segment table of this phase by warp 0:
-        // [shared down groups (several tokens)] + routed gate/up groups
-        const int n_sd = kOutRows ? 0 : n_sg;
+        // [shared down groups (several token groups)] + routed gate/up groups
+        const int n_sd = all_x ? 0 : n_sg;
         if (warp == 0) {
             const int n_rg = union_warp<MT>(u, T, k, E, a.err);
             __syncwarp();
@@ -1286,6 +1242,24 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                     const int g = s - n_sd, e = u.gexp[g];
                     return item_cost<kRW, nd>(H, min(MT, u.off[e] + u.cnt[e] - u.gpos[g]));
                 });
+        } else if (all_x) {
+            // one token group: the shared expert's gate/up for the staged tokens, on the other warps
+            // beside the routing (this CTA's even share of the F row pairs, two rows a step through a
+            // ring of twice the slots: a warp holds about one item, its steps nearly all in flight)
+            constexpr int R2 = P_GU * kRW / 2;
+            const int s_lo = (int)((long long)F * blockIdx.x / gridDim.x);
+            const int s_hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
+            auto rows_of = [&](int j, Rows<2>& r) { gateup_rows(r, (size_t)E * F + j); };
+            auto vecs_of = [&](int, VecSet<MT>& v) {
+                v.m = T;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) v.vi[t] = t;
+            };
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) { gateup_finish(j, P, v, tot); };
+            const int first = s_lo + warp - 1;
+            const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 2) / (kLayerWarps - 1) : 0;
+            stream_rows<MT, 2, R2, nd>(first, kLayerWarps - 1, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of,
+                                       vecs_of, fin);
         }
         __syncthreads();
         stamp(a, 12);
@@ -1438,15 +1412,16 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             else static_cast<float*>(a.out)[n] = acc;
         }
     } else {
-        // several tokens: routed down rows, one partial output row per pair (routing weight applied)
-        const int nseg = u.gpre[E];  // routed groups
+        // several tokens: routed down rows, one partial output row per pair (routing weight applied);
+        // for one token group first the shared expert's down rows (its h at P + t, weight 1)
+        const int n_sdc = all_x ? 1 : 0;
+        const int nseg = n_sdc + u.gpre[E];
+        auto seg_e = [&](int s) { return s < n_sdc ? E : u.gexp[s - n_sdc]; };
+        auto seg_p0 = [&](int s) { return s < n_sdc ? P : u.gpos[s - n_sdc]; };
+        auto seg_m = [&](int s) { return s < n_sdc ? T : min(MT, u.off[seg_e(s)] + u.cnt[seg_e(s)] - seg_p0(s)); };
         if (warp == 0)
             seg_build_warp(
-                u, nseg, [&](int) { return H / kRW; },
-                [&](int s) {
-                    const int e = u.gexp[s];
-                    return item_cost<kRW, nd>(F, min(MT, u.off[e] + u.cnt[e] - u.gpos[s]));
-                });
+                u, nseg, [&](int) { return H / kRW; }, [&](int s) { return item_cost<kRW, nd>(F, seg_m(s)); });
         __syncthreads();
         const SegTable st{u.seg_i, u.seg_c, u.seg_cost, u.tmp, nseg};
         int lo, hi;
@@ -1454,8 +1429,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         for (int s = 0; s < nseg; ++s) {
             const int s_lo = max(lo, st.ipre[s]), s_hi = min(hi, st.ipre[s + 1]);
             if (s_lo >= s_hi) continue;
-            const int e = u.gexp[s], p0 = u.gpos[s];
-            const int m = min(MT, u.off[e] + u.cnt[e] - p0);
+            const bool shared = s < n_sdc;
+            const int e = seg_e(s), p0 = seg_p0(s);
+            const int m = seg_m(s);
             __syncthreads();
             stage_h(m, p0);
             __syncthreads();
@@ -1471,8 +1447,8 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
                 const int n0 = kRW * (j - base);
                 rows_out(v, tot, [&](int r, int t, float y) {
-                    if (COLI_IN_BOUNDS(p0 + t < P && n0 + r < H, a.err)) {
-                        const float wt = u.w[u.perm[p0 + t]];
+                    if (COLI_IN_BOUNDS(p0 + t < (shared ? P + T : P) && n0 + r < H, a.err)) {
+                        const float wt = shared ? 1.0f : u.w[u.perm[p0 + t]];
                         a.y[(size_t)(p0 + t) * H + n0 + r] = wt * y;
                     }
                 });
