@@ -399,7 +399,8 @@ LayerPlan layer_plan(int T, int H, int F, int E, int k, int nd)
 {
     LayerPlan p;
     if (T < 1 || T > kLayerMaxT) return p;
-    const int rows_per_cta = 2 * ((H / 2 + kMinLayerSms - 1) / kMinLayerSms);
+    const int ru = layer_rows(1, nd);  // one token: output rows are split in units of ru rows
+    const int rows_per_cta = ru * ((H / ru + kMinLayerSms - 1) / kMinLayerSms);
     auto fits = [&](int MT, bool rows) {
         const LayerSmem ls = layer_smem(T, H, F, E, k, MT, rows, rows_per_cta, nd);
         if (ls.bytes > (size_t)kSmemBudget) return false;

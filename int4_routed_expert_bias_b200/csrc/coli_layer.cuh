@@ -397,10 +397,10 @@ struct LayerSmem {
     int ring_slots;
 };
 
-// Rows per engine step: four for groups of several tokens whose activations
-// take at most two digits (each activation load then serves four rows; their
-// ring fits beside the staged vectors), else two.
-__host__ __device__ constexpr int layer_rows(int MT, int nd) { return MT > 1 && nd <= 2 ? 4 : 2; }
+// Rows per engine step: four (each activation load then serves four rows),
+// except for groups of several tokens of three-digit activations, whose four
+// staged vectors leave no room for the four-row ring.
+__host__ __device__ constexpr int layer_rows(int MT, int nd) { return MT == 1 || nd <= 2 ? 4 : 2; }
 
 // Ring slots per warp (steps in flight + 1): deeper when fewer activation
 // vectors are staged, shallower for the four-row slots.
@@ -1089,8 +1089,9 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
 
     // ======================= phase B: top-k, union, routed gate/up =======================
     const int S1 = k + 1;  // one token: slots (routed in order, shared last)
-    const int pr_lo = (int)((long long)(H / 2) * blockIdx.x / gridDim.x);  // one token: this CTA's output row pairs
-    const int npr = (int)((long long)(H / 2) * (blockIdx.x + 1) / gridDim.x) - pr_lo;
+    // one token: this CTA's output rows, units pr_lo .. pr_lo + npr - 1 of kRW rows each
+    const int pr_lo = (int)((long long)(H / kRW) * blockIdx.x / gridDim.x);
+    const int npr = (int)((long long)(H / kRW) * (blockIdx.x + 1) / gridDim.x) - pr_lo;
     const int npc = a.n_pieces == 0 ? (gH.per_lane + kPieceChunks - 1) / kPieceChunks : a.n_pieces;
     float* s_logit = reinterpret_cast<float*>(lsm + ls.logit);
     if constexpr (kOutRows) {
@@ -1148,33 +1149,34 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             __syncthreads();
         };
         {
-            const int s_lo = (int)((long long)F * blockIdx.x / gridDim.x);
-            const int s_hi = (int)((long long)F * (blockIdx.x + 1) / gridDim.x);
-            auto rows_of = [&](int j, Rows<2>& r) { gateup_rows(r, (size_t)E * F + j); };
+            const int s_lo = (int)((long long)(F / kHP) * blockIdx.x / gridDim.x);
+            const int s_hi = (int)((long long)(F / kHP) * (blockIdx.x + 1) / gridDim.x);
+            auto rows_of = [&](int j, Rows<kRW>& r) { gateup_rows(r, (size_t)E * F + kHP * j); };
             auto vecs_of = [&](int, VecSet<MT>& v) {
                 v.m = 1;
 #pragma unroll
                 for (int t = 0; t < MT; ++t) v.vi[t] = 0;
             };
-            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) { gateup_finish(j, P, v, tot); };
+            auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) { gateup_finish(kHP * j, P, v, tot); };
             const int first = s_lo + warp;
             const int nj = first < s_hi ? (s_hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-            stream_rows<MT, 2, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
-                                         fin, route_hook);
+            stream_rows<MT, kRW, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
+                                           fin, route_hook);
         }
         stamp(a, 14);
         stamp(a, 4);
-        // routed gate/up: the kept experts x F rows, equal cost, an even split
+        // routed gate/up: the kept experts x F / kHP items, equal cost, an even split
         const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
-        const int total = n_kept * F;
+        const int fi = F / kHP;  // items per expert
+        const int total = n_kept * fi;
         const int lo = (int)((long long)total * blockIdx.x / gridDim.x);
         const int hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
-        const FastDiv div_f(F, total);
-        auto rows_of = [&](int j, Rows<2>& r) {
+        const FastDiv div_f(fi, total);
+        auto rows_of = [&](int j, Rows<kRW>& r) {
             const int g = div_f(j);
             int e = u.gexp[g];
             if (!COLI_IN_BOUNDS(e >= 0 && e < E, a.err)) e = 0;
-            gateup_rows(r, (size_t)e * F + (j - g * F));
+            gateup_rows(r, (size_t)e * F + kHP * (j - g * fi));
         };
         auto vecs_of = [&](int, VecSet<MT>& v) {
             v.m = 1;
@@ -1183,13 +1185,14 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.vi[t] = 0;
             }
         };
-        auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[2][MT]) {
+        auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
             const int g = div_f(j);
-            gateup_finish(j - g * F, g, v, tot);
+            gateup_finish(kHP * (j - g * fi), g, v, tot);
         };
         const int first = lo + warp;
         const int nj = first < hi ? (hi - first + kLayerWarps - 1) / kLayerWarps : 0;
-        stream_rows<MT, 2, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of, fin);
+        stream_rows<MT, kRW, P_GU, nd>(first, kLayerWarps, nj, gH.per_lane, gH.nch, xs, xcorr, ring, rows_of, vecs_of,
+                                       fin);
     } else {
         const bool scored_here = all_x;  // the kernel scored the tokens (npc partial pieces per score)
         if (scored_here) {
@@ -1357,15 +1360,15 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         // depend on it), the h vectors are staged after it
         const int S = S1;
         // item j = (slot g = j / npr: the g-th kept expert in ascending order, the shared expert
-        // at g = n_kept; row pair)
+        // at g = n_kept; unit of kRW output rows)
         const int n_kept = reinterpret_cast<const int*>(u.tmp)[0];
         const int n_slots = n_kept + 1;
         const FastDiv div_pr(npr, (long long)npr * n_slots);
-        auto rows_of = [&](int j, Rows<2>& r) {
+        auto rows_of = [&](int j, Rows<kRW>& r) {
             const int slot = div_pr(j), pr = pr_lo + (j - slot * npr);
             int e = slot < n_kept ? u.gexp[slot] : E;
-            if (!COLI_IN_BOUNDS(e >= 0 && e <= E && 2 * pr + 1 < H, a.err)) e = 0;
-            down_rows(r, (size_t)e * H + 2 * pr);
+            if (!COLI_IN_BOUNDS(e >= 0 && e <= E && kRW * pr + kRW - 1 < H, a.err)) e = 0;
+            down_rows(r, (size_t)e * H + kRW * pr);
         };
         auto vecs_of = [&](int j, VecSet<MT>& v) {
             const int slot = div_pr(j);
@@ -1375,11 +1378,10 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
                 v.vi[t] = slot;
             }
         };
-        auto fin = [&](int j, const VecSet<MT>&, const float (&tot)[2][MT]) {
+        auto fin = [&](int j, const VecSet<MT>& v, const float (&tot)[kRW][MT]) {
             const int slot = div_pr(j), pl = j - slot * npr;
             const int col = slot < n_kept ? slot : k;  // the shared expert's column is k
-            const float y = warp_sum2(tot[0][0], tot[1][0]);  // lane 0: row 2 pl, lane 16: row 2 pl + 1
-            if ((lane & 15) == 0) ypart[(2 * pl + (lane >> 4)) * S + col] = y;
+            rows_out(v, tot, [&](int r, int, float y) { ypart[(kRW * pl + r) * S + col] = y; });
         };
         auto hook = [&]() {
             grid_barrier(bar, deadline, a.err);
@@ -1398,16 +1400,16 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
         const int total = npr * n_slots;
         const int first = warp;
         const int nj = first < total ? (total - first + kLayerWarps - 1) / kLayerWarps : 0;
-        stream_rows<MT, 2, P_DN, nd>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of, fin,
-                                     hook);
+        stream_rows<MT, kRW, P_DN, nd>(first, kLayerWarps, nj, gF.per_lane, gF.nch, hs, hcorr, ring, rows_of, vecs_of,
+                                       fin, hook);
         __syncthreads();
         stamp(a, 8);
-        for (int i = threadIdx.x; i < 2 * npr; i += kLayerThreads) {
+        for (int i = threadIdx.x; i < kRW * npr; i += kLayerThreads) {
             float acc = 0.f;
             for (int j = 0; j < k; ++j)
                 if (u.ipos[j] >= 0) acc = fmaf(u.w[j], ypart[i * S + u.ipos[j]], acc);
             acc += ypart[i * S + k];
-            const int n = 2 * pr_lo + i;
+            const int n = kRW * pr_lo + i;
             if constexpr (kOutBf16) static_cast<uint16_t*>(a.out)[n] = float_to_bf16_bits(acc);
             else static_cast<float*>(a.out)[n] = acc;
         }
