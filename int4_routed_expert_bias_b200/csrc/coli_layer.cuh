@@ -104,6 +104,19 @@ __device__ __forceinline__ void grid_barrier(GridBar& b, unsigned long long dead
     __syncthreads();
 }
 
+// Warp sums of four values: the sum of a lands on lanes 0-7 (read on lane 0),
+// of b on lane 8, of c on lane 16, of d on lane 24; six shuffles.
+__device__ __forceinline__ float warp_sum4(float a, float b, float c, float d)
+{
+    const bool h16 = (threadIdx.x & 16) != 0, h8 = (threadIdx.x & 8) != 0;
+    const float v1 = (h16 ? c : a) + __shfl_xor_sync(0xFFFFFFFFu, h16 ? a : c, 16);
+    const float v2 = (h16 ? d : b) + __shfl_xor_sync(0xFFFFFFFFu, h16 ? b : d, 16);
+    float v = (h8 ? v2 : v1) + __shfl_xor_sync(0xFFFFFFFFu, h8 ? v1 : v2, 8);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
 // ---------------------------------------------------------------------------
 // the rolling int4 row-pair engine
 
