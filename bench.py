@@ -519,10 +519,12 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         entry["layer_tflops"] = layer_flops / (ms_per_step * 1e-3) / 1e12
         entry["layer_frac_of_bf16_sustained"] = entry["layer_tflops"] / bf16_sust
 
-    # end to end through the public call with host buffers: pinned x in, out back
+    # end to end through the C-ABI call with host buffers (coli_moe_forward_host): every step copies
+    # that step's pinned activations in and the output back, and the host waits for the result
     if not args.no_e2e:
         n_e2e = 16 if prefill else min(max(steps, 64), 1024)
         xh = [torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).pin_memory() for x in xs_host]
+        xh = [t.view(torch.bfloat16) if xdt == torch.bfloat16 else t for t in xh]
         xin = torch.empty_like(xs[0])
         oh = torch.empty((c.T, c.H), dtype=odt).pin_memory()
         barrier(world)
@@ -530,17 +532,14 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s)
         for i in range(n_e2e):
-            src = xh[i % G]
-            xin.view(torch.int16 if xdt == torch.bfloat16 else xdt).copy_(src, non_blocking=True)
-            coli.moe_forward(layers[i % N_LAYERS], xin, out, ws)
-            oh.copy_(out, non_blocking=True)
+            coli.moe_forward_host(layers[i % N_LAYERS], xh[i % G], xin, oh, out, ws)
             s.synchronize()
         e1.record(s)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world, torch)
         entry["e2e"] = {"value": job_throughput(world, n_e2e, c.T, ems), "unit": "tokens/s",
                         "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
-                        "steps": n_e2e, "host_sync_per_step": True}
+                        "steps": n_e2e, "host_sync_per_step": True, "call": "coli_moe_forward_host"}
 
     # the oracle on this machine's host cores, bounded sample, rank 0 at N=1 only
     if world == 1 and not args.no_cpu:

@@ -253,6 +253,27 @@ COLI_API coli_status coli_moe_forward_noalloc(const coli_moe_layer* layer, const
                                               int T, void* out, coli_dtype ot, int32_t* topk_idx_out,
                                               float* topk_w_out, cudaStream_t stream);
 
+/*
+ * The layer end to end from host memory: the per-token path of
+ * coli_moe_forward (Korean getting-started page, section 토큰당 처리 경로)
+ * with the activations read from and the output written to host buffers, the
+ * way an engine that keeps its token state on the host would call it.  Three
+ * steps are enqueued on stream, in order: x_host [T, H] (dtype xt) is copied
+ * into the caller's device buffer x_dev [T, H]; coli_moe_forward runs on
+ * x_dev into the caller's device buffer out_dev [T, H] (dtype ot) with the
+ * given workspace; out_dev is copied to out_host [T, H].  Host buffers should
+ * be page-locked (cudaHostAlloc / cudaHostRegister) for the copies to be
+ * asynchronous; the caller owns all five buffers, and out_host holds the
+ * result once the stream has reached the end of the call (e.g. after
+ * cudaStreamSynchronize).  Every argument (those of coli_moe_forward, the two
+ * host pointers and the workspace size) is checked before anything is
+ * enqueued; COLI_ERR_CUDA if a copy cannot be enqueued.  T == 0 enqueues
+ * nothing.
+ */
+COLI_API coli_status coli_moe_forward_host(const coli_moe_layer* layer, const void* x_host, void* x_dev,
+                                           coli_dtype xt, int T, void* out_host, void* out_dev, coli_dtype ot,
+                                           void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 COLI_API const char* coli_status_string(coli_status status);
 COLI_API const char* coli_last_error(void);
 

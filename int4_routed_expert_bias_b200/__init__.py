@@ -40,6 +40,8 @@ _lib.coli_moe_forward.restype = _i
 _lib.coli_moe_forward.argtypes = [_p, _p, _i, _i, _p, _i, _p, ctypes.c_size_t, _p, _p, _p]
 _lib.coli_moe_forward_noalloc.restype = _i
 _lib.coli_moe_forward_noalloc.argtypes = [_p, _p, _i, _i, _p, _i, _p, _p, _p]
+_lib.coli_moe_forward_host.restype = _i
+_lib.coli_moe_forward_host.argtypes = [_p, _p, _p, _i, _i, _p, _p, _i, _p, ctypes.c_size_t, _p]
 _lib.coli_moe_profile_next.restype = _i
 _lib.coli_moe_profile_next.argtypes = [_p, _i]
 _lib.coli_status_string.restype = ctypes.c_char_p
@@ -161,6 +163,17 @@ def moe_forward(layer, x, out, workspace, topk_idx_out=None, topk_w_out=None, st
     _check(_lib.coli_moe_forward(layer.ref, _ptr(x), _dtype_code(x), T, _ptr(out), _dtype_code(out),
                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _ptr(topk_idx_out), _ptr(topk_w_out), _stream(stream)))
+
+
+def moe_forward_host(layer, x_host, x_dev, out_host, out_dev, workspace, stream=None):
+    """The layer from host memory: x_host (pinned CPU tensor) is copied into
+    x_dev, the layer runs into out_dev, and out_dev is copied into out_host
+    (pinned CPU tensor), all on the stream; see include/coli.h."""
+    if x_host.dtype != x_dev.dtype or out_host.dtype != out_dev.dtype:
+        raise ValueError("host and device buffers must have the same dtype")
+    _check(_lib.coli_moe_forward_host(layer.ref, _ptr(x_host), _ptr(x_dev), _dtype_code(x_dev), x_host.shape[0],
+                                      _ptr(out_host), _ptr(out_dev), _dtype_code(out_dev), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def moe_forward_noalloc(layer, x, out, topk_idx_out=None, topk_w_out=None, stream=None):

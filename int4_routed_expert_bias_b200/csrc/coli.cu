@@ -794,6 +794,26 @@ coli_status noalloc_scratch(void** out)
 
 }  // namespace
 
+extern "C" coli_status coli_moe_forward_host(const coli_moe_layer* L, const void* x_host, void* x_dev, coli_dtype xt,
+                                             int T, void* out_host, void* out_dev, coli_dtype ot, void* workspace,
+                                             size_t ws_bytes, cudaStream_t stream)
+{
+    coli_status st = check_call(L, x_dev, xt, T, out_dev, ot, nullptr, nullptr);
+    if (st != COLI_OK || T == 0) return st;
+    if (!x_host || !out_host || !workspace) return fail(COLI_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(workspace, 256)) return fail(COLI_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    const size_t need = coli_moe_workspace_size(L, T);
+    if (ws_bytes < need) return fail(COLI_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
+    const size_t n = (size_t)T * L->hidden;
+    const size_t xb = n * (xt == COLI_BF16 ? 2 : 4), ob = n * (ot == COLI_BF16 ? 2 : 4);
+    cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "input copy");
+    if ((st = coli_moe_forward(L, x_dev, xt, T, out_dev, ot, workspace, ws_bytes, nullptr, nullptr, stream)) != COLI_OK)
+        return st;
+    e = cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, stream);
+    return e == cudaSuccess ? COLI_OK : cuda_fail(e, "output copy");
+}
+
 extern "C" coli_status coli_moe_forward_noalloc(const coli_moe_layer* L, const void* x, coli_dtype xt, int T,
                                                 void* out, coli_dtype ot, int32_t* topk_idx_out,
                                                 float* topk_w_out, cudaStream_t stream)

@@ -131,6 +131,25 @@ def test_forward_rejects_bad_calls(coli):
     assert "workspace" in coli.last_error()
 
 
+def _fwd_host(coli, s, T=1, xh=1 << 21, xd=1 << 20, oh=1 << 21, od=1 << 20, ws=1 << 20, ws_bytes=1 << 30):
+    L = coli.lib()
+    return L.coli_moe_forward_host(ctypes.byref(s), xh, xd, 0, T, oh, od, 0, ws, ws_bytes, None)
+
+
+def test_forward_host_rejects_bad_calls(coli):
+    # every argument is checked before anything is enqueued (no CUDA call is made for these)
+    s = _layer(coli)
+    assert _fwd_host(coli, s, xh=0) == 1
+    assert _fwd_host(coli, s, oh=0) == 1
+    assert _fwd_host(coli, s, xd=0) == 1
+    assert _fwd_host(coli, s, od=(1 << 20) + 4) == 1
+    assert _fwd_host(coli, s, ws=(1 << 20) + 16) == 1
+    assert _fwd_host(coli, s, T=-1) == 1
+    need = coli.lib().coli_moe_workspace_size(ctypes.byref(s), 1)
+    assert _fwd_host(coli, s, ws_bytes=need - 1) == 3
+    assert _fwd_host(coli, s, T=0, xh=0, oh=0, xd=0, od=0, ws=0, ws_bytes=0) == 0
+
+
 def test_empty_forward_is_ok_without_launching(coli):
     assert _fwd(coli, _layer(coli), T=0, x=0, out=0, ws=0, ws_bytes=0) == 0
 
