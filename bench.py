@@ -71,6 +71,8 @@ def parse(argv=None):
     ap.add_argument("--experts", type=int, default=0,
                     help="routed experts per layer (0 = the workload's; profiling: fewer, same per-call bytes)")
     ap.add_argument("--replays", type=int, default=0, help="timed replays of the K steps (0 = sized to ~0.3 s)")
+    ap.add_argument("--lookahead", action="store_true",
+                    help="also time decode batch 1 with the router-lookahead prefetch of the next layer")
     ap.add_argument("--int8", action="store_true",
                     help="also time the integer-activation variant of the chosen --config (always with no --config)")
     ap.add_argument("--top-p", type=float, default=0.0,
@@ -344,10 +346,13 @@ def path_dtype(path, act_int8=False, x_bf16=False):
     return "f32"
 
 
-def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sampler_index, top_p=0.0, act_int8=False):
+def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sampler_index, top_p=0.0, act_int8=False,
+                     lookahead=False):
     """Time one workload; returns the fields of its benchmark entry.  top_p > 0
     runs the layer with adaptive expert top-p routing; act_int8 the
-    integer-activation variant (int8 activations per 32 values)."""
+    integer-activation variant (int8 activations per 32 values); lookahead names
+    each call's next layer (the resident layers are called in order) for the
+    router-lookahead prefetch."""
     hbm_peak, bf16_peak, bf16_sust, peak_kind = peaks
     routers, layers = [], []
     for l in range(N_LAYERS):
@@ -357,6 +362,9 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         layers.append(coli.Layer(c.H, c.F, c.E, c.k, c.routed_scale, torch.from_numpy(w_router).cuda(),
                                  torch.from_numpy(sel_bias).cuda(), b["gate_q"], b["gate_s"], b["up_q"],
                                  b["up_s"], b["down_q"], b["down_s"], top_p=top_p, act_int8=act_int8))
+    if lookahead:
+        for l in range(N_LAYERS):
+            layers[l].set_prefetch_next(layers[(l + 1) % N_LAYERS])
     path = coli.moe_path(layers[0], c.T)
 
     # activation pool: G distinct (step, layer) batches, G a multiple of the layer count
@@ -467,7 +475,7 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
     layer_gbs = layer_alg / (ms_per_step * 1e-3) / 1e9
     kname, kstage, kfile = DOMINANT[path]
     # the committed summaries are of the default kernel on the plain top-k routing
-    traffic = traffic_from_profiles(kfile, c.name) if not (top_p or act_int8) else None
+    traffic = traffic_from_profiles(kfile, c.name) if not (top_p or act_int8 or lookahead) else None
     prefill = path == "prefill"
     if prefill:
         # dominant kernel: the gate/up grouped GEMM, 2 * (pairs + shared) * 2F * H flops
@@ -502,8 +510,10 @@ def measure_workload(args, torch, coli, c, res, seed, world, rank, peaks, sample
         roofline["traffic_over_alg"] = traffic / alg if alg else None
     expert_alg = float(np.mean((U + 1) * c.expert_bytes))  # selected experts' int4 + scales only
     entry = {"workload": workload_desc(c) + (f", adaptive expert top-p {top_p}" if top_p else "") +
-             (", int8 activations (integer-dot variant)" if act_int8 else ""),
+             (", int8 activations (integer-dot variant)" if act_int8 else "") +
+             (", router-lookahead prefetch of the next layer's router and shared expert" if lookahead else ""),
              "tokens_per_call": c.T, "path": path, "value": value, "top_p": top_p, "act_int8": bool(act_int8),
+             "lookahead": bool(lookahead),
              "dtype": path_dtype(path, act_int8, c.x_dtype == "bf16"),
              "unit": "tokens/s", "steps": steps, "timed_replays": R, "ms_per_step": ms_per_step,
              "ms_per_step_p10": percentile(ms_max, 10) / steps, "ms_per_step_p90": percentile(ms_max, 90) / steps,
@@ -606,6 +616,14 @@ def run_ours(args):
                                 torch.cuda.current_device(), top_p=args.top_p or 0.7)
         torch.cuda.empty_cache()
 
+    look = None
+    if not args.config or args.lookahead:
+        # decode batch 1 naming each call's next layer: the router-lookahead prefetch of its router and
+        # shared expert during the routing of this call
+        look = measure_workload(args, torch, coli, cfg_of(1), res, seed, world, rank, peaks,
+                                torch.cuda.current_device(), lookahead=True)
+        torch.cuda.empty_cache()
+
     head_cfg = cfgs[0]
     head, c = entries[head_cfg], cfg_of(head_cfg)
     extra = {"parallelism": f"replicas x{world}", "path": head["path"], "mean_union_U": head["mean_union_U"],
@@ -616,10 +634,12 @@ def run_ours(args):
              "expert_alg_bytes_per_call": head["expert_alg_bytes_per_call"],
              "expert_frac_of_hbm_peak": head["expert_frac_of_hbm_peak"], "stage_ms": head["stage_ms"],
              "timing": "median of the timed replays of exactly K steps (CUDA events, max over ranks)"}
-    if len(cfgs) > 1 or topp is not None or int8:
+    if len(cfgs) > 1 or topp is not None or int8 or look is not None:
         extra["per_workload"] = {cfg_of(k).name: entries[k] for k in cfgs[1:]}
         if topp is not None:
             extra["per_workload"][f"{cfg_of(1).name}-topp{topp['top_p']}"] = topp
+        if look is not None:
+            extra["per_workload"][f"{cfg_of(1).name}-lookahead"] = look
         for k, ent in int8.items():
             extra["per_workload"][f"{cfg_of(k).name}-int8"] = ent
     line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": head["steps"],

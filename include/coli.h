@@ -62,7 +62,7 @@ typedef enum { COLI_F32 = 0, COLI_BF16 = 1 } coli_dtype;
 
 /* One MoE layer.  Expert index n_experts is the shared expert, so every
  * expert array holds n_experts + 1 experts, expert-major. */
-typedef struct {
+typedef struct coli_moe_layer {
     int hidden;            /* H, e.g. 6144 */
     int ffn;               /* F, expert width, e.g. 2048 */
     int n_experts;         /* E routed experts, e.g. 256 */
@@ -79,6 +79,8 @@ typedef struct {
     const float* down_s;   /* [E+1, H, F/64] */
     float top_p;           /* adaptive expert top-p: 0 (or >= 1) = plain top-k; see coli_moe_forward */
     int act_int8;          /* 1: integer-activation variant (int8 activations per 32); 0: default; see coli_moe_forward */
+    const struct coli_moe_layer* prefetch_next; /* the layer the next call runs, for the router-lookahead
+                                                   prefetch, or NULL; see coli_moe_forward */
 } coli_moe_layer;
 
 /*
@@ -164,6 +166,16 @@ COLI_API size_t coli_moe_status_word_offset(const coli_moe_layer* layer, int T);
  * The quantisation rule is this library's reading.  Batches of up to 64 tokens
  * only: a larger batch with act_int8 set returns COLI_ERR_UNSUPPORTED.  out is
  * written as fp32 or bf16 (round to nearest even).
+ * Router-lookahead prefetch ("Colibri 完全ガイド", section Router-Lookahead
+ * プリフェッチ: the next layer's experts are fetched while the current layer
+ * computes): when layer->prefetch_next is set (checked like layer itself), a
+ * one-token call asks the L2 cache for that layer's router weights, selection
+ * bias and shared expert (weights and scales) while it routes its own token,
+ * when the memory is otherwise idle, so that the next call finds them in L2.
+ * The next layer's routed experts are not predicted: their router input is the
+ * next layer's activations, which this call does not have (this library's
+ * reading).  The results are unchanged; batches of more than one token ignore
+ * the field.
  * x [T, H] dtype xt; out [T, H] dtype ot; workspace of at least
  * coli_moe_workspace_size(layer, T) bytes, contents undefined on entry and on
  * exit apart from the status word (coli_moe_status_word_offset), not shared by

@@ -66,7 +66,7 @@ class _LayerStruct(ctypes.Structure):
                 ("w_router", _p), ("sel_bias", _p),
                 ("gate_q", _p), ("up_q", _p), ("down_q", _p),
                 ("gate_s", _p), ("up_s", _p), ("down_s", _p), ("top_p", ctypes.c_float),
-                ("act_int8", ctypes.c_int)]
+                ("act_int8", ctypes.c_int), ("prefetch_next", _p)]
 
 
 def lib():
@@ -123,6 +123,12 @@ class Layer:
     @property
     def ref(self):
         return ctypes.byref(self.struct)
+
+    def set_prefetch_next(self, other):
+        """Name the layer the next call runs (None: none), for the router-lookahead
+        prefetch of its router and shared expert; see include/coli.h."""
+        self._next = other  # keeps the other layer's struct alive while it is named here
+        self.struct.prefetch_next = None if other is None else ctypes.addressof(other.struct)
 
 
 def router_topk(x, w_router, sel_bias, k, routed_scale, topk_idx, topk_w, stream=None):

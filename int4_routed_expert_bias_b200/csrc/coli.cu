@@ -245,7 +245,7 @@ Workspace layout(void* base, int T, int H, int F, int E, int k)
     return w;
 }
 
-coli_status check_layer(const coli_moe_layer* L, int T)
+coli_status check_layer_fields(const coli_moe_layer* L, int T)
 {
     if (!L) return fail(COLI_ERR_INVALID_ARG, "layer is NULL");
     coli_status st = check_sizes(T, L->hidden, L->n_experts, L->top_k);
@@ -264,6 +264,47 @@ coli_status check_layer(const coli_moe_layer* L, int T)
         if (!aligned(ptrs[i], i == 1 ? 4 : 16)) return fail(COLI_ERR_INVALID_ARG, "layer.%s is not 16-byte aligned", names[i]);
     }
     return COLI_OK;
+}
+
+// The layer's fields, and those of the layer named for the router-lookahead prefetch (not followed further).
+coli_status check_layer(const coli_moe_layer* L, int T)
+{
+    coli_status st = check_layer_fields(L, T);
+    if (st != COLI_OK || !L->prefetch_next) return st;
+    if ((st = check_layer_fields(L->prefetch_next, 1)) != COLI_OK) {
+        char why[256];
+        snprintf(why, sizeof why, "%s", coli_last_error());
+        return fail(st, "prefetch_next: %s", why);
+    }
+    return COLI_OK;
+}
+
+// Byte ranges of layer N that the router-lookahead prefetch asks L2 for: its router weights and
+// selection bias, and its shared expert's three matrices and their scales (16-byte aligned inside).
+int lookahead_ranges(const coli_moe_layer* N, const unsigned char** base, unsigned long long* bytes)
+{
+    const size_t H = N->hidden, F = N->ffn, E = N->n_experts;
+    const struct {
+        const void* p;
+        size_t off, n;
+    } r[] = {{N->w_router, 0, E * H * 4},
+             {N->sel_bias, 0, E * 4},
+             {N->gate_q, E * F * (H / 2), F * (H / 2)},
+             {N->up_q, E * F * (H / 2), F * (H / 2)},
+             {N->down_q, E * H * (F / 2), H * (F / 2)},
+             {N->gate_s, E * F * (H / kGroup) * 4, F * (H / kGroup) * 4},
+             {N->up_s, E * F * (H / kGroup) * 4, F * (H / kGroup) * 4},
+             {N->down_s, E * H * (F / kGroup) * 4, H * (F / kGroup) * 4}};
+    int n = 0;
+    for (const auto& x : r) {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(x.p) + x.off;
+        const uintptr_t lo = (a + 15) & ~(uintptr_t)15, hi = (a + x.n) & ~(uintptr_t)15;
+        if (hi <= lo || n == kMaxPrefetch) continue;
+        base[n] = reinterpret_cast<const unsigned char*>(lo);
+        bytes[n] = hi - lo;
+        ++n;
+    }
+    return n;
 }
 
 // Argument checks of a layer call other than its workspace (host only).
@@ -597,6 +638,7 @@ coli_status coli_moe_forward(const coli_moe_layer* L, const void* x, coli_dtype 
         LayerArgs la{L->w_router, L->sel_bias, L->gate_q, L->gate_s, L->up_q, L->up_s, L->down_q, L->down_s,
                      H, F, E, k, T, L->routed_scale, x, out, w.logits, fused_router ? 0 : 1, idx, wt, w.h,
                      w.partial, w.ctl + 3, wait_limit(kBarrierNs), L->top_p, g_stamps.load()};
+        if (pl.out_rows && L->prefetch_next) la.pf_n = lookahead_ranges(L->prefetch_next, la.pf_base, la.pf_bytes);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(dev->sms);
         cfg.blockDim = dim3(layer_threads(pl.MT));

@@ -214,6 +214,12 @@ __device__ __forceinline__ uint64_t l2_evict_first()
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
+// Asks the L2 cache for the bytes [p, p + n) (p and n multiples of 16); no completion to wait for.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* p, uint32_t n)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ void cp_async16_s(uint32_t smem, const void* gmem, uint64_t pol)
 {
     asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem), "l"(gmem), "l"(pol)
@@ -363,6 +369,8 @@ __device__ __forceinline__ void stream_rows(int j0, int js, int nj, int per_lane
 // ---------------------------------------------------------------------------
 // layer arguments and shared-memory layout
 
+constexpr int kMaxPrefetch = 8;  // router weights, selection bias, the shared expert's 3 matrices and 3 scale arrays
+
 struct LayerArgs {
     const float* w_router;  // [E, H]
     const float* sel_bias;  // [E]
@@ -386,6 +394,10 @@ struct LayerArgs {
     unsigned long long wait_ns;  // limit of each grid-barrier wait
     float top_p;            // adaptive expert top-p (0: plain top-k)
     unsigned long long* stamps;  // optional [gridDim.x, kStamps] globaltimer stamps per CTA (test hook)
+    // router lookahead: byte ranges of the next layer to bring into L2 (pf_n of them, one token only)
+    const unsigned char* pf_base[kMaxPrefetch];
+    unsigned long long pf_bytes[kMaxPrefetch];
+    int pf_n;
 };
 
 constexpr int kStamps = 16;
@@ -1397,6 +1409,17 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
             rows_out(v, tot, [&](int r, int, float y) { ypart[(kRW * pl + r) * S + col] = y; });
         };
         auto hook = [&]() {
+            if (a.pf_n > 0 && warp == kLayerWarps - 1) {
+                // router lookahead, while the blocks meet and stage h (the memory is otherwise idle then):
+                // this CTA's share of each range of the next layer, up to 4 KB per lane request
+                for (int r = 0; r < a.pf_n && r < kMaxPrefetch; ++r) {
+                    const unsigned long long B = a.pf_bytes[r];
+                    const unsigned long long lo = (B * blockIdx.x / gridDim.x) & ~15ull;
+                    const unsigned long long hi = (B * (blockIdx.x + 1) / gridDim.x) & ~15ull;
+                    for (unsigned long long off = lo + 4096ull * lane; off < hi; off += 32ull * 4096)
+                        l2_prefetch_bulk(a.pf_base[r] + off, (uint32_t)(hi - off < 4096ull ? hi - off : 4096ull));
+                }
+            }
             grid_barrier(bar, deadline, a.err);
             stamp(a, 6);
             // h of the g-th kept expert sits at position g, the shared expert's at P (= k)

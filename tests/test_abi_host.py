@@ -150,6 +150,18 @@ def test_forward_host_rejects_bad_calls(coli):
     assert _fwd_host(coli, s, T=0, xh=0, oh=0, xd=0, od=0, ws=0, ws_bytes=0) == 0
 
 
+def test_forward_checks_the_lookahead_layer(coli):
+    s, n = _layer(coli), _layer(coli, gate_q=0)
+    s.prefetch_next = ctypes.addressof(n)
+    assert _fwd(coli, s) == 1
+    assert "prefetch_next" in coli.last_error()
+    n2 = _layer(coli, group=32)
+    s.prefetch_next = ctypes.addressof(n2)
+    assert _fwd(coli, s) == 2
+    s.prefetch_next = ctypes.addressof(s)  # a layer may name itself: the check does not follow the chain
+    assert _fwd(coli, s, ws_bytes=1) == 3
+
+
 def test_empty_forward_is_ok_without_launching(coli):
     assert _fwd(coli, _layer(coli), T=0, x=0, out=0, ws=0, ws_bytes=0) == 0
 
