@@ -673,20 +673,25 @@ __device__ __forceinline__ int last_le(const V* a, int n, long long x)
 }
 
 // This CTA's items of the phase: those whose start cost lies in
-// [C b / G, C (b + 1) / G).
+// [C b / G, C (b + 1) / G).  The quotients are taken in double precision,
+// exact here (the costs stay far below 2^53 / G, and a ceiling quotient that
+// is not an integer is at least 1 / cost from one), without the slow 64-bit
+// integer division; a boundary shared by two CTAs is the same expression in
+// both.
 __device__ __forceinline__ void seg_cta_range(const SegTable& st, int& lo, int& hi)
 {
     const long long C = st.cpre[st.nseg];
     auto first = [&](long long x) -> int {
         const int s = last_le(st.cpre, st.nseg, x);
         if (s >= st.nseg) return st.ipre[st.nseg];
-        const long long c = st.cost[s] > 0 ? st.cost[s] : 1;
-        const long long r = (x - st.cpre[s] + c - 1) / c;
+        const int c = st.cost[s] > 0 ? st.cost[s] : 1;
+        const long long r = (long long)ceil((double)(x - st.cpre[s]) / (double)c);
         const long long n = st.ipre[s + 1] - st.ipre[s];
         return st.ipre[s] + (int)(r < n ? r : n);
     };
-    lo = first(C * (long long)blockIdx.x / gridDim.x);
-    hi = first(C * (long long)(blockIdx.x + 1) / gridDim.x);
+    const double G = (double)gridDim.x;
+    lo = first((long long)floor((double)C * blockIdx.x / G));
+    hi = first((long long)floor((double)C * (blockIdx.x + 1) / G));
 }
 
 // Union tables in shared memory (every CTA computes the same ones).
