@@ -260,14 +260,15 @@ def run_reference(args):
 
     budget = 60.0
     max_calls = max(1, args.steps)
-    # warm-up: one call, untimed (page-in of the oracle and the inputs)
-    time_oracle_calls(c_sample, xs, routers, get_expert, 0.0, min(1, args.warmup))
+    # warm-up: W untimed calls (page-in of the oracle and the inputs; one bounded call each)
+    warm = max(args.warmup, 3)
+    time_oracle_calls(c_sample, xs, routers, get_expert, float("inf"), warm)
     n, spent, cores = time_oracle_calls(c_sample, xs, routers, get_expert, budget, max_calls)
     tok_s = n * c_sample.T / spent
     sample = (f"{n} layer calls of {c_sample.T} token(s) (of {c.T} per call), the oracle's f64 plain loops, "
               f"stopped after {budget:.0f} s of oracle time")
     line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": n, "warmup": min(1, args.warmup), "ms_per_step": 1e3 * spent / n,
+            "steps": n, "warmup": warm, "ms_per_step": 1e3 * spent / n,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_block(c, len(xs)),
             "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
