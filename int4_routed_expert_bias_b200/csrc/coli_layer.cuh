@@ -938,7 +938,7 @@ moe_layer_kernel(const LayerArgs a, const LayerSmem ls)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StageGeom gH = stage_geom(H), gF = stage_geom(F);
     float4* xs = reinterpret_cast<float4*>(lsm + ls.x_off);
-    constexpr int kPieceChunks = MT == 1 ? 2 : 1;  // router chunks per lane per piece
+    constexpr int kPieceChunks = 2;  // router chunks per lane per piece
     // staged vectors as digit planes (16-byte units per vector)
     const int xvs = digit_vec_units(H, nd);
     const int hvs = digit_vec_units(F, nd);
