@@ -176,57 +176,6 @@ __device__ __forceinline__ void stage_vectors_part(int n, Load4 load, const Stag
     }
 }
 
-// Stage n vectors of K values (rows of src, fp32 or bf16): vector t is row
-// row0 + t of src, or row tbl[t] / tdiv when tbl is given.  Same layout and
-// arithmetic as stage_vectors_part, in a compact form for the paths that run
-// once per call: one copy of the code serves every call site, four loads in
-// flight per thread.  Threads tid = 0 .. nthr-1 (whole warps) share the work.
-static __device__ __noinline__ void stage_rows(const void* __restrict__ src, int bf16, int K, int n, int row0,
-                                        const int* tbl, int tdiv, float4* xs, float* corr, int tid, int nthr)
-{
-    const StageGeom g = stage_geom(K);
-    const int per_vec = g.nch * 8;
-    const int total = n * per_vec;
-    const size_t row_bytes = (size_t)K * (bf16 ? 2 : 4);
-    for (int base = 0; base < total; base += 4 * nthr) {
-        float4 v[4];
-        int tt[4], rem[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int idx = base + r * nthr + tid;
-            v[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-            tt[r] = 0;
-            rem[r] = 0;
-            if (idx < total) {
-                const int t = idx / per_vec;
-                const int re = idx - t * per_vec;
-                tt[r] = t;
-                rem[r] = re;
-                const int row = tbl ? tbl[t] / tdiv : row0 + t;
-                const char* rp = static_cast<const char*>(src) + (size_t)row * row_bytes;
-                const int i = (re >> 3) * kChunkK + (re & 7) * 4;
-                v[r] = bf16 ? load_act4<true>(rp, i) : load_act4<false>(rp, i);
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const bool valid = base + r * nthr + tid < total;
-            const int c = rem[r] >> 3, j = rem[r] & 7;
-            if (valid)
-                xs[(size_t)tt[r] * g.f4 + ((c >> 5) * 8 + j) * 32 + ((c & 31) ^ j)] =
-                    make_float4(v[r].y, v[r].x, v[r].w, v[r].z);
-            float odd = v[r].y + v[r].w, even = v[r].x + v[r].z;
-            odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 1);
-            even += __shfl_xor_sync(0xFFFFFFFFu, even, 1);
-            odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 2);
-            even += __shfl_xor_sync(0xFFFFFFFFu, even, 2);
-            odd += __shfl_xor_sync(0xFFFFFFFFu, odd, 4);
-            even += __shfl_xor_sync(0xFFFFFFFFu, even, 4);
-            if (valid && j == 0) corr[tt[r] * g.nch + c] = fmaf(-24.f, odd, -264.f * even);
-        }
-    }
-}
-
 // ---------------------------------------------------------------------------
 // Integer-dot form of the one-vector products.
 //

@@ -481,21 +481,6 @@ __host__ __device__ inline LayerSmem layer_smem(int T, int H, int F, int E, int 
     return s;
 }
 
-// ---------------------------------------------------------------------------
-// small block-level helpers (every thread of the block calls them)
-
-// Segment lookup: the segment s with pre[s] <= x < pre[s + 1] (pre ascending, pre[0] = 0).
-__device__ __forceinline__ int seg_find(const int* pre, int nseg, long long x)
-{
-    int lo = 0, hi = nseg - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if ((long long)pre[mid] <= x) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
 }  // namespace coli
 
 namespace coli {
