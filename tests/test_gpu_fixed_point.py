@@ -8,8 +8,8 @@ same call alike).  Blocks whose largest magnitude is below 2^-100 contribute
 nothing.  These cases put a block of zeros, a block of values near 1e-30 and
 one near 1e-33 (either side of that cut-off), a block with one value 50 times
 its neighbours' scale and a block spanning twenty
-binary orders into x, for one token, a 4-token group and 33 tokens (token
-groups), in fp32 and bf16, with every one-token and several-token stream
+binary orders into x, for one token, one group of 2, 3 or 4 tokens, 5 tokens
+(a full group and one of a single token) and 33 tokens, in fp32 and bf16, with every one-token and several-token stream
 shape the kernel has (four rows per step; two for several fp32 tokens).  The
 output is held to the decode tolerance and the routing must be exact.
 """
@@ -41,8 +41,9 @@ def _experts(rng, H, F, E):
     return ex
 
 
-@pytest.mark.parametrize("T,xdt,path", [(1, "f32", "single"), (1, "bf16", "single"), (4, "f32", "decode"),
-                                        (4, "bf16", "decode"), (33, "f32", "decode"), (33, "bf16", "decode")])
+@pytest.mark.parametrize("T,xdt,path", [(1, "f32", "single"), (1, "bf16", "single"), (2, "bf16", "decode"),
+                                        (3, "bf16", "decode"), (4, "f32", "decode"), (4, "bf16", "decode"),
+                                        (5, "bf16", "decode"), (33, "f32", "decode"), (33, "bf16", "decode")])
 def test_edge_blocks_match_the_oracle(env, T, xdt, path):
     coli, torch = env
     H, F, E, k = 1024, 512, 64, 8
